@@ -1,0 +1,107 @@
+"""Plain fp64 CPU oracle for causal scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package; the library in
+``causal_attention_sdpa_b200`` never does, and this package never imports it.
+
+The arithmetic lives in ``oracle.c`` (plain row-by-row loops in double
+precision, OpenMP over heads).  This module only compiles it with gcc and
+marshals numpy arrays through ctypes.
+
+Definition followed (restated, not copied): "NanoGPT Speedrun baseline",
+section "El Mecanismo de Atencion" -- softmax(QK^T / sqrt(d_k)) V with
+Attn_ij = 0 for j > i -- and, for the optional window, the long/short
+sliding-window attention item of the modded-nanogpt README's technique list.
+The backward pass is the exact gradient of sum(O * dO).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so with gcc (-O2, OpenMP, strict IEEE)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        L = ctypes.c_long
+        lib.oracle_attn_fwd.argtypes = [dp, dp, dp, L, L, L, ctypes.c_double, L,
+                                        dp, dp, ctypes.c_int]
+        lib.oracle_attn_fwd.restype = ctypes.c_int
+        lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, L, L, L, ctypes.c_double, L,
+                                        dp, dp, dp, dp, ctypes.c_int]
+        lib.oracle_attn_bwd.restype = ctypes.c_int
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _as_f64(x) -> np.ndarray:
+    """Accept numpy arrays or torch CPU tensors (any float dtype) -> C-contiguous float64."""
+    if hasattr(x, "detach"):  # torch tensor; bf16 widens exactly to fp32 and fp64
+        x = x.detach().to("cpu").float().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def attn_fwd(q, k, v, scale: float, window: int = 0, nthreads: int = 0):
+    """Forward pass.  q, k, v: [..., T, D].  Returns (O [..., T, D], lse [..., T]) in fp64."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    if not (q.shape == k.shape == v.shape) or q.ndim < 2:
+        raise ValueError("q, k, v must share one shape [..., T, D]")
+    *lead, T, D = q.shape
+    NH = int(np.prod(lead)) if lead else 1
+    o = np.zeros_like(q)
+    lse = np.zeros(tuple(lead) + (T,), dtype=np.float64)
+    rc = _load().oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), NH, T, D, float(scale),
+                                 int(window), _ptr(o), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd failed with code {rc}")
+    return o, lse
+
+
+def attn_bwd(q, k, v, dO, scale: float, window: int = 0, nthreads: int = 0):
+    """Backward pass of sum(O * dO).  Returns (dQ, dK, dV, Delta) in fp64."""
+    q, k, v, dO = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dO)
+    if not (q.shape == k.shape == v.shape == dO.shape) or q.ndim < 2:
+        raise ValueError("q, k, v, dO must share one shape [..., T, D]")
+    *lead, T, D = q.shape
+    NH = int(np.prod(lead)) if lead else 1
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    delta = np.zeros(tuple(lead) + (T,), dtype=np.float64)
+    rc = _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), NH, T, D,
+                                 float(scale), int(window), _ptr(dq), _ptr(dk),
+                                 _ptr(dv), _ptr(delta), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_bwd failed with code {rc}")
+    return dq, dk, dv, delta
+

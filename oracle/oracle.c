@@ -1,0 +1,191 @@
+/*
+ * Plain fp64 CPU oracle for causal multi-head scaled-dot-product attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file: only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark use it.  It shares no code, header or constant with the CUDA
+ * library.
+ *
+ * What it computes is the plain definition, written out row by row with no
+ * tiling, no online rescaling and no reordering beyond what the definition
+ * states:
+ *
+ *   Forward ("NanoGPT Speedrun baseline", section "El Mecanismo de Atencion",
+ *   the Attn(Q,K,V) = softmax(QK^T / sqrt(d_k)) V equation and the mask rule
+ *   Attn_ij = 0 for j > i; the boolean triu(diagonal=1) mask of "Un GPT desde
+ *   cero + nanoGPT", Laboratorio L2.1, True = blocked):
+ *     S_ij  = scale * sum_d Q_id K_jd            for visible (i, j)
+ *     m_i   = max_j S_ij
+ *     lse_i = m_i + ln sum_j exp(S_ij - m_i)     (natural log)
+ *     P_ij  = exp(S_ij - lse_i)                  (0 where not visible)
+ *     O_i   = sum_j P_ij V_j
+ *   Key j is visible to query i iff j <= i and (window <= 0 or j > i - window);
+ *   the window is the sliding-window variant named in the modded-nanogpt
+ *   README's technique list (long/short sliding-window attention).  Masked
+ *   entries are -inf before the softmax, so every row renormalises over its
+ *   visible keys.
+ *
+ *   Backward: the exact gradient of L = sum(O * dO) with respect to Q, K, V
+ *   (the pages only call loss.backward(); the gradient of the definition
+ *   above is the one reading):
+ *     dV_j    = sum_i P_ij dO_i
+ *     dP_ij   = dO_i . V_j
+ *     Delta_i = sum_j P_ij dP_ij
+ *     dS_ij   = P_ij (dP_ij - Delta_i)
+ *     dQ_i    = scale * sum_j dS_ij K_j
+ *     dK_j    = scale * sum_i dS_ij Q_i
+ *
+ * Layout: contiguous [NH, T, D] row-major doubles (NH = B*H heads as an extra
+ * batch dimension, as in the GPT-2 lecture's attention module).  Each head is
+ * independent; heads are spread over OpenMP threads.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static int visible(long i, long j, long window) {
+    if (j > i) return 0;
+    if (window > 0 && j <= i - window) return 0;
+    return 1;
+}
+
+/* Row i of the softmax: fills p[0..i] (p[j] = 0 where not visible), returns lse. */
+static double softmax_row(const double* q, const double* k, long T, long D,
+                          double scale, long window, long i, double* p) {
+    (void)T;
+    double m = -INFINITY;
+    for (long j = 0; j <= i; ++j) {
+        if (!visible(i, j, window)) { p[j] = -INFINITY; continue; }
+        double s = 0.0;
+        for (long d = 0; d < D; ++d) s += q[i * D + d] * k[j * D + d];
+        s *= scale;
+        p[j] = s;
+        if (s > m) m = s;
+    }
+    double sum = 0.0;
+    for (long j = 0; j <= i; ++j)
+        if (visible(i, j, window)) sum += exp(p[j] - m);
+    double lse = m + log(sum);
+    for (long j = 0; j <= i; ++j)
+        p[j] = visible(i, j, window) ? exp(p[j] - lse) : 0.0;
+    return lse;
+}
+
+static void fwd_head(const double* q, const double* k, const double* v,
+                     long T, long D, double scale, long window,
+                     double* o, double* lse, double* p) {
+    for (long i = 0; i < T; ++i) {
+        lse[i] = softmax_row(q, k, T, D, scale, window, i, p);
+        for (long d = 0; d < D; ++d) {
+            double acc = 0.0;
+            for (long j = 0; j <= i; ++j) acc += p[j] * v[j * D + d];
+            o[i * D + d] = acc;
+        }
+    }
+}
+
+static void bwd_head(const double* q, const double* k, const double* v,
+                     const double* dO, long T, long D, double scale, long window,
+                     double* dq, double* dk, double* dv, double* delta,
+                     double* p, double* dp) {
+    memset(dk, 0, sizeof(double) * T * D);
+    memset(dv, 0, sizeof(double) * T * D);
+    for (long i = 0; i < T; ++i) {
+        softmax_row(q, k, T, D, scale, window, i, p);
+        /* dV_j += P_ij dO_i ; dP_ij = dO_i . V_j */
+        for (long j = 0; j <= i; ++j) {
+            if (p[j] != 0.0)
+                for (long d = 0; d < D; ++d) dv[j * D + d] += p[j] * dO[i * D + d];
+            double s = 0.0;
+            if (visible(i, j, window))
+                for (long d = 0; d < D; ++d) s += dO[i * D + d] * v[j * D + d];
+            dp[j] = s;
+        }
+        double del = 0.0;
+        for (long j = 0; j <= i; ++j) del += p[j] * dp[j];
+        delta[i] = del;
+        for (long d = 0; d < D; ++d) dq[i * D + d] = 0.0;
+        for (long j = 0; j <= i; ++j) {
+            double ds = p[j] * (dp[j] - del);
+            if (ds == 0.0) continue;
+            for (long d = 0; d < D; ++d) {
+                dq[i * D + d] += scale * ds * k[j * D + d];
+                dk[j * D + d] += scale * ds * q[i * D + d];
+            }
+        }
+    }
+}
+
+static int bad_args(long NH, long T, long D) {
+    return NH < 0 || T < 0 || D <= 0;
+}
+
+/* Returns 0 on success, 1 on bad arguments, 2 on allocation failure. */
+int oracle_attn_fwd(const double* q, const double* k, const double* v,
+                    long NH, long T, long D, double scale, long window,
+                    double* o, double* lse, int nthreads) {
+    if (bad_args(NH, T, D)) return 1;
+    if (NH == 0 || T == 0) return 0;
+    int fail = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads) reduction(| : fail)
+#endif
+    {
+        double* p = (double*)malloc(sizeof(double) * T);
+        if (!p) fail = 1;
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (long h = 0; h < NH; ++h) {
+            if (!p) continue;
+            fwd_head(q + h * T * D, k + h * T * D, v + h * T * D, T, D, scale,
+                     window, o + h * T * D, lse + h * T, p);
+        }
+        free(p);
+    }
+    (void)nthreads;
+    return fail ? 2 : 0;
+}
+
+int oracle_attn_bwd(const double* q, const double* k, const double* v,
+                    const double* dO, long NH, long T, long D, double scale,
+                    long window, double* dq, double* dk, double* dv,
+                    double* delta, int nthreads) {
+    if (bad_args(NH, T, D)) return 1;
+    if (NH == 0 || T == 0) return 0;
+    int fail = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads) reduction(| : fail)
+#endif
+    {
+        double* p = (double*)malloc(sizeof(double) * T);
+        double* dp = (double*)malloc(sizeof(double) * T);
+        if (!p || !dp) fail = 1;
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (long h = 0; h < NH; ++h) {
+            if (!p || !dp) continue;
+            bwd_head(q + h * T * D, k + h * T * D, v + h * T * D, dO + h * T * D,
+                     T, D, scale, window, dq + h * T * D, dk + h * T * D,
+                     dv + h * T * D, delta + h * T, p, dp);
+        }
+        free(p);
+        free(dp);
+    }
+    (void)nthreads;
+    return fail ? 2 : 0;
+}
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
