@@ -1,0 +1,348 @@
+#!/usr/bin/env python
+"""Benchmark: causal attention forward + backward TFLOP/s on B200.
+
+One step = one forward pass (gpt_attn_fwd) and one backward pass
+(gpt_attn_bwd_delta -> gpt_attn_bwd_grads -> gpt_attn_bwd_dq_convert) over
+one batch of the GPT-2 124M attention workload at micro-batch 64
+(B=64, H=12, T=1024, D=64, causal, scale 1/8), seeded N(0,1) bf16 inputs.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  `value` counts 7*B*H*T^2*D flops per step
+(forward 2*B*H*T^2*D, backward 2.5x that) on every rank, divided by the
+slowest rank's device time for the K timed steps.  Under torchrun each rank
+drives one GPU with its own copy of the workload (weak scaling; attention has
+no exchange step).  `--impl reference` times the fp64 CPU oracle on a bounded
+sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=workloads.HEADLINE.index,
+                    help="workload number (1-5); the default is the headline shape")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "causal_attention_sdpa_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, units: float):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    # bytes were captured on e["units"] (b*h*T^2 pairs-equivalent units); scale to this launch
+    return e["dram_bytes"] * units / e["units"]
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.samples = []
+        if self.proc is None:
+            return False
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 8:
+                self.samples.append(parts)
+        return False
+
+    def summary(self):
+        if not getattr(self, "samples", None):
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm = [float(p[1]) for p in self.samples if p[1].replace(".", "").isdigit()]
+        mx = [float(p[2]) for p in self.samples if p[2].replace(".", "").isdigit()]
+        reasons = sorted({names[i] for p in self.samples for i in range(4) if p[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def oracle_sample(w, q, k, v, do, n_heads):
+    import oracle
+    heads = workloads.sample_heads(w.B, w.H, n_heads, seed=1)
+    sel = lambda t: __import__("torch").stack([t[b, h] for b, h in heads])
+    qs, ks, vs, dos = sel(q), sel(k), sel(v), sel(do)
+    t0 = time.perf_counter()
+    oracle.attn_fwd(qs, ks, vs, w.scale, w.window)
+    oracle.attn_bwd(qs, ks, vs, dos, w.scale, w.window)
+    dt = time.perf_counter() - t0
+    flops = workloads.fwd_bwd_flops(1, len(heads), w.T, w.D, w.window)
+    return flops, dt, len(heads), oracle.max_threads()
+
+
+def run_reference(args, w, rank):
+    """The CPU oracle, timed on the host cores on a bounded sample of the workload."""
+    if rank != 0:
+        return
+    import oracle
+    q, k, v, do = workloads.workload_inputs(w)
+    cores = oracle.max_threads()
+    n = min(w.B * w.H, max(1, cores) * 4)
+    for _ in range(args.warmup):
+        oracle_sample(w, q, k, v, do, n)
+    tot_f, tot_t = 0.0, 0.0
+    for _ in range(args.steps):
+        f, t, nh, cores = oracle_sample(w, q, k, v, do, n)
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12
+    sample = (f"{nh} of {w.B * w.H} heads (b,h) of the workload per step, fwd+bwd, fp64 oracle "
+              f"(OpenMP over heads)")
+    line = {
+        "impl": "reference", "metric": "causal attention fwd+bwd TFLOP/s", "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.describe(), "B": w.B, "H": w.H, "T": w.T, "D": w.D, "window": w.window,
+            "scale": w.scale, "qk_norm": w.qk_norm, "seed": w.seed,
+            "l2": "inputs larger than L2 (4 x %.0f MB bf16 > 126 MB), no flush" % (w.B * w.H * w.T * w.D * 2 / 1e6),
+            "flop_count": ("7*B*H*T^2*D (fwd 2*B*H*T^2*D, bwd 2.5x)" if w.window <= 0 or w.window >= w.T
+                           else "algorithmic: 4*D per visible pair fwd, 10*D bwd")}
+
+
+def main():
+    args = parse_args()
+    w = workloads.BY_INDEX[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, w, rank)
+
+    import torch
+    import causal_attention_sdpa_b200 as ga
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    ga.lib()
+
+    # Host copies (pinned) for the end-to-end leg; device copies for the kernel leg.
+    q_h, k_h, v_h, do_h = workloads.workload_inputs(w)
+    q_h, k_h, v_h, do_h = (t.pin_memory() for t in (q_h, k_h, v_h, do_h))
+    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
+    B, H, T, D = w.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(ga.gpt_attn_bwd_workspace_bytes(B, H, T, D), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ga.gpt_attn_fwd(q, k, v, scale=w.scale, window=w.window, o=o, lse=lse, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        ga.gpt_attn_bwd_delta(o, lse, do, ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        ga.gpt_attn_bwd_grads(q, k, v, do, dk, dv, ws, scale=w.scale, window=w.window, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        ga.gpt_attn_bwd_dq_convert(dq, ws, stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    status = ga.gpt_attn_check(stream)
+    if status != ga.GPT_ATTN_OK:
+        raise RuntimeError(f"warm-up failed: {ga.status_string(status)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(local) as clk:
+        time.sleep(0.25)   # let the sampler start before the timed region
+        barrier()
+        for i in range(args.steps):
+            step(evs[i])
+        barrier()
+    status = ga.gpt_attn_check(stream)
+    if status != ga.GPT_ATTN_OK:
+        raise RuntimeError(f"timed steps failed: {ga.status_string(status)}")
+    total_ms = evs[0][0].elapsed_time(evs[-1][4])
+    per_kernel = {name: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps
+                  for i, name in enumerate(("attn_fwd_kernel", "attn_bwd_prep_kernel", "attn_bwd_kernel",
+                                            "attn_dq_convert_kernel"))}
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = t.item()
+
+    flops_step = workloads.fwd_bwd_flops(B, H, T, D, w.window)
+    value = flops_step * world * args.steps / (total_ms / 1e3) / 1e12
+
+    # ---- end to end: pinned host buffers in and out through the public API, copies timed
+    e2e = None
+    if not args.no_e2e:
+        o_h = torch.empty_like(q_h).pin_memory()
+        lse_h = torch.empty((B, H, T), dtype=torch.float32).pin_memory()
+        dq_h, dk_h, dv_h = (torch.empty_like(q_h).pin_memory() for _ in range(3))
+        e_steps = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            for d_, h_ in ((q, q_h), (k, k_h), (v, v_h), (do, do_h)):
+                d_.copy_(h_, non_blocking=True)
+            ga.gpt_attn_fwd(q, k, v, scale=w.scale, window=w.window, o=o, lse=lse, stream=stream)
+            ga.gpt_attn_bwd(q, k, v, o, lse, do, scale=w.scale, window=w.window, dq=dq, dk=dk, dv=dv,
+                            workspace=ws, stream=stream)
+            for h_, d_ in ((o_h, o), (lse_h, lse), (dq_h, dq), (dk_h, dk), (dv_h, dv)):
+                h_.copy_(d_, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = t.item()
+        n_el = B * H * T * D
+        e2e = {"value": flops_step * world * e_steps / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 4 * n_el * 2, "d2h_bytes_per_step": 4 * n_el * 2 + B * H * T * 4,
+               "steps": e_steps}
+        status = ga.gpt_attn_check(stream)
+        if status != ga.GPT_ATTN_OK:
+            raise RuntimeError(f"end-to-end steps failed: {ga.status_string(status)}")
+
+    if rank != 0:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    peaks = load_peaks()
+    fwd_f = workloads.fwd_flops(B, H, T, D, w.window)
+    bwd_f = flops_step - fwd_f
+    kflops = {"attn_fwd_kernel": fwd_f, "attn_bwd_kernel": bwd_f}
+    dominant = max(kflops, key=lambda n: per_kernel[n])
+    achieved = kflops[dominant] / (per_kernel[dominant] / 1e3) / 1e12
+    roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                "peak_source": f"{peaks['source']} burst dense bf16",
+                "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                      if peaks.get("bf16_tflops_sustained") else None),
+                "traffic": recorded_traffic(dominant, B * H)}
+    n_el = B * H * T * D
+    prep_bytes = 2 * n_el * 2 + 4 * n_el + B * H * T * 4 * 3
+    kernels = {n: {"ms": per_kernel[n]} for n in per_kernel}
+    kernels["attn_fwd_kernel"]["tflops"] = fwd_f / (per_kernel["attn_fwd_kernel"] / 1e3) / 1e12
+    kernels["attn_bwd_kernel"]["tflops"] = bwd_f / (per_kernel["attn_bwd_kernel"] / 1e3) / 1e12
+    kernels["attn_bwd_prep_kernel"]["gbs"] = prep_bytes / (per_kernel["attn_bwd_prep_kernel"] / 1e3) / 1e9
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        import oracle  # the CPU baseline leg: oracle only
+        cores = oracle.max_threads()
+        f, t, nh, cores = oracle_sample(w, q_h, k_h, v_h, do_h, min(B * H, max(1, cores) * 24))
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{nh} of {B * H} heads (b,h) of the workload, fwd+bwd, fp64, {t:.1f} s wall"}
+
+    line = {
+        "metric": "causal attention fwd+bwd TFLOP/s", "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(w),
+        "pct_of_peak": value / world / peaks["bf16_tflops"],
+        "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": 4 * args.steps, "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,198 @@
+"""Python binding of the gpt_attn C ABI (libgpt_attn.so, built in-tree for sm_100a).
+
+Argument marshalling only: every step of the attention computation runs in the
+CUDA kernels behind the C ABI.  PyTorch supplies device memory and streams.
+There is no CPU or library fallback: if the shared library is missing or
+cannot be loaded, importing the functions raises.
+
+Entry points (same names as the C ABI, see include/gpt_attn.h):
+  gpt_attn_fwd(q, k, v, scale=None, window=0, o=None, lse=None, stream=None) -> (o, lse)
+  gpt_attn_bwd(q, k, v, o, lse, dO, scale=None, window=0, dq=None, dk=None, dv=None,
+               workspace=None, stream=None) -> (dq, dk, dv)
+  gpt_attn_bwd_workspace_bytes(B, H, T, D) -> int
+  gpt_attn_check(stream=None) -> int
+  gpt_attn_status_string(status) -> str
+Tensors are bf16 contiguous [B, H, T, D] on the GPU; lse is fp32 [B, H, T].
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgpt_attn.so")
+
+GPT_ATTN_OK = 0
+GPT_ATTN_ERR_NULL = 1
+GPT_ATTN_ERR_SHAPE = 2
+GPT_ATTN_ERR_UNSUPPORTED_D = 3
+GPT_ATTN_ERR_ALIGN = 4
+GPT_ATTN_ERR_CUDA = 5
+GPT_ATTN_ERR_TIMEOUT = 6
+GPT_ATTN_ERR_WORKSPACE = 7
+
+EXPORTED = ("gpt_attn_fwd", "gpt_attn_bwd", "gpt_attn_bwd_workspace_bytes", "gpt_attn_bwd_delta",
+            "gpt_attn_bwd_grads", "gpt_attn_bwd_dq_convert", "gpt_attn_check", "gpt_attn_status_string",
+            "gpt_attn_debug_wait_timeout")
+
+_lib = None
+
+
+class GptAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgpt_attn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m causal_attention_sdpa_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.gpt_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.gpt_attn_fwd.restype = i
+        L.gpt_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+        L.gpt_attn_bwd.restype = i
+        L.gpt_attn_bwd_delta.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
+        L.gpt_attn_bwd_delta.restype = i
+        L.gpt_attn_bwd_grads.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+        L.gpt_attn_bwd_grads.restype = i
+        L.gpt_attn_bwd_dq_convert.argtypes = [vp, i, i, i, i, vp, sz, vp]
+        L.gpt_attn_bwd_dq_convert.restype = i
+        L.gpt_attn_bwd_workspace_bytes.argtypes = [i, i, i, i]
+        L.gpt_attn_bwd_workspace_bytes.restype = sz
+        L.gpt_attn_check.argtypes = [vp]
+        L.gpt_attn_check.restype = i
+        L.gpt_attn_status_string.argtypes = [i]
+        L.gpt_attn_status_string.restype = ctypes.c_char_p
+        L.gpt_attn_debug_wait_timeout.argtypes = [i, vp]
+        L.gpt_attn_debug_wait_timeout.restype = i
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().gpt_attn_status_string(int(status)).decode()
+
+
+gpt_attn_status_string = status_string
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _check_bf16(name, t, shape):
+    import torch
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(shape)}")
+
+
+def gpt_attn_fwd(q, k, v, scale=None, window=0, o=None, lse=None, stream=None):
+    """Forward pass; returns (o, lse).  Asynchronous on `stream` (default: current)."""
+    import torch
+    B, H, T, D = q.shape
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_bf16(n, t, q.shape)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    _check_bf16("o", o, q.shape)
+    rc = lib().gpt_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, D, float(scale),
+                            int(window), _stream_handle(stream))
+    if rc != GPT_ATTN_OK:
+        raise GptAttnError(rc, "gpt_attn_fwd")
+    return o, lse
+
+
+def gpt_attn_bwd_workspace_bytes(B, H, T, D) -> int:
+    return int(lib().gpt_attn_bwd_workspace_bytes(int(B), int(H), int(T), int(D)))
+
+
+def gpt_attn_bwd(q, k, v, o, lse, dO, scale=None, window=0, dq=None, dk=None, dv=None, workspace=None,
+                 stream=None):
+    """Backward pass of sum(O * dO); returns (dq, dk, dv).  Asynchronous on `stream`."""
+    import torch
+    B, H, T, D = q.shape
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO)):
+        _check_bf16(n, t, q.shape)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    need = gpt_attn_bwd_workspace_bytes(B, H, T, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().gpt_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk),
+                            _ptr(dv), B, H, T, D, float(scale), int(window), _ptr(workspace), ws_bytes,
+                            _stream_handle(stream))
+    if rc != GPT_ATTN_OK:
+        raise GptAttnError(rc, "gpt_attn_bwd")
+    return dq, dk, dv
+
+
+def _ws(workspace, q):
+    import torch
+    B, H, T, D = q.shape
+    if workspace is None:
+        workspace = torch.empty(max(gpt_attn_bwd_workspace_bytes(B, H, T, D), 16), dtype=torch.uint8,
+                                device=q.device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def gpt_attn_bwd_delta(o, lse, dO, workspace, stream=None):
+    """Stage 1 of the backward pass (Delta, scaled lse, zeroed dQ accumulator)."""
+    B, H, T, D = o.shape
+    ws, nbytes = _ws(workspace, o)
+    rc = lib().gpt_attn_bwd_delta(_ptr(o), _ptr(lse), _ptr(dO), B, H, T, D, _ptr(ws), nbytes,
+                                  _stream_handle(stream))
+    if rc != GPT_ATTN_OK:
+        raise GptAttnError(rc, "gpt_attn_bwd_delta")
+    return ws
+
+
+def gpt_attn_bwd_grads(q, k, v, dO, dk, dv, workspace, scale=None, window=0, stream=None):
+    """Stage 2 of the backward pass (dK, dV written; dQ accumulated in the workspace)."""
+    B, H, T, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    ws, nbytes = _ws(workspace, q)
+    rc = lib().gpt_attn_bwd_grads(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dk), _ptr(dv), B, H, T, D,
+                                  float(scale), int(window), _ptr(ws), nbytes, _stream_handle(stream))
+    if rc != GPT_ATTN_OK:
+        raise GptAttnError(rc, "gpt_attn_bwd_grads")
+
+
+def gpt_attn_bwd_dq_convert(dq, workspace, stream=None):
+    """Stage 3 of the backward pass (bf16 dQ from the fp32 accumulator)."""
+    B, H, T, D = dq.shape
+    ws, nbytes = _ws(workspace, dq)
+    rc = lib().gpt_attn_bwd_dq_convert(_ptr(dq), B, H, T, D, _ptr(ws), nbytes, _stream_handle(stream))
+    if rc != GPT_ATTN_OK:
+        raise GptAttnError(rc, "gpt_attn_bwd_dq_convert")
+
+
+def gpt_attn_check(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return int(lib().gpt_attn_check(_stream_handle(stream)))
+
+
+def gpt_attn_debug_wait_timeout(timeout_us: int, stream=None) -> int:
+    return int(lib().gpt_attn_debug_wait_timeout(int(timeout_us), _stream_handle(stream)))

@@ -1,0 +1,439 @@
+// Backward pass of L = sum(O * dO) for causal / sliding-window attention.
+//
+// The gradient is the exact one of the forward definition
+// ("NanoGPT Speedrun baseline", section "El Mecanismo de Atencion"):
+//   P = softmax(scale * Q K^T) (blocked keys 0), dV = P^T dO, dP = dO V^T,
+//   Delta_i = dO_i . O_i, dS = P * (dP - Delta), dQ = scale dS K, dK = scale dS^T Q.
+// The pages only call loss.backward(); the decomposition through Delta is an
+// algebraic identity of this gradient, not a different result.
+//
+// Three kernels run in order on the caller's stream:
+//   attn_bwd_prep_kernel   Delta_i = dO_i . O_i and lse*log2(e) into padded
+//                          per-head rows of the workspace; zeroes the fp32 dQ
+//                          accumulator.  HBM-bound.
+//   attn_bwd_kernel<D>     one CTA per (batch*head, 128-key tile); K and V stay
+//                          in shared memory, query tiles stream through a TMA
+//                          ring.  Per query tile, five tcgen05 MMAs:
+//                            S^T  = K Q^T          (TMEM)
+//                            dP^T = V dO^T         (TMEM)
+//                            dV  += P^T dO         (P^T read from TMEM)
+//                            dK  += dS^T Q         (dS^T from shared memory)
+//                            dQ   = dS K           (same shared tile, MN-major)
+//                          dQ is added into the fp32 accumulator with vector
+//                          red.global.add by a dedicated warpgroup.
+//   attn_dq_convert_kernel fp32 accumulator -> bf16 dQ.
+// The score scale is folded into dS before its bf16 rounding, so dK and dQ
+// need no epilogue scaling.
+#pragma once
+
+#include "attn_fwd.cuh"
+
+namespace gpt_attn {
+
+constexpr int kBwdThreads = 320;     // 10 warps
+
+struct BwdParams {
+    const float* lse2;      // [BH, T_pad]  lse * log2(e); +inf past T
+    const float* delta;     // [BH, T_pad]  dO_i . O_i;    0 past T
+    float* dq_acc;          // [BH, T, D]   fp32, zeroed by the prep kernel
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    int T;
+    int T_pad;
+    int BH;
+    int n_tiles;
+    int window;
+    float scale_log2;       // scale * log2(e)
+    float scale;
+    uint64_t timeout_ns;
+};
+
+template <int D>
+struct BwdCfg {
+    static constexpr int kStages = (D == 64) ? 2 : 1;      // Q/dO ring depth (shared-memory bound)
+    static constexpr int kTileBytes = kTile * D * 2;
+    static constexpr uint32_t kColS = 0;                    // S^T, then P^T (bf16) over its first 64 columns
+    static constexpr uint32_t kColDP = 128;                 // dP^T
+    static constexpr uint32_t kColDV = 256;
+    static constexpr uint32_t kColDK = 256 + D;
+    static constexpr uint32_t kColDQ = (D == 64) ? 384 : 0; // D = 128: dQ reuses the S^T columns
+    static constexpr bool kDqAliasesS = (D != 64);
+};
+
+template <int D>
+struct BwdSmem {
+    using C = BwdCfg<D>;
+    alignas(1024) uint8_t k[C::kTileBytes];
+    alignas(1024) uint8_t v[C::kTileBytes];
+    alignas(1024) uint8_t q[C::kStages][C::kTileBytes];
+    alignas(1024) uint8_t dout[C::kStages][C::kTileBytes];
+    alignas(1024) uint8_t ds[kTile * kTile * 2];           // dS^T bf16 [key][query], two 64-query halves
+    alignas(16) float lse2[C::kStages][kTile];
+    alignas(16) float delta[C::kStages][kTile];
+    uint64_t bar_kv;
+    uint64_t bar_qdo_full[C::kStages];
+    uint64_t bar_qdo_empty[C::kStages];
+    uint64_t bar_s_full;
+    uint64_t bar_dp_full;
+    uint64_t bar_p_full;
+    uint64_t bar_ds_full;
+    uint64_t bar_dv_done;
+    uint64_t bar_ds_empty;
+    uint64_t bar_dq_full;
+    uint64_t bar_dq_empty;
+    uint64_t bar_dkdv_full;
+    uint64_t bar_drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// Query tiles that see at least one key of key tile kt: [kt, qt_hi].
+__device__ __forceinline__ int bwd_last_query_tile(int kt, int n_tiles, int window) {
+    if (window <= 0) return n_tiles - 1;
+    const long last = (long)kt * kTile + kTile - 1 + window - 1;   // last query that sees a key of the tile
+    const long t = last / kTile;
+    return t < n_tiles - 1 ? (int)t : n_tiles - 1;
+}
+
+__global__ void attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                                     const float* __restrict__ lse, float* __restrict__ lse2,
+                                     float* __restrict__ delta, float* __restrict__ dq_acc, int T, int T_pad,
+                                     long long total_rows_pad, int D) {
+    // One warp per padded row.
+    const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= total_rows_pad) return;
+    const long long bh = row / T_pad;
+    const int t = (int)(row - bh * T_pad);
+    if (t >= T) {
+        if (lane == 0) {
+            lse2[row] = INFINITY;
+            delta[row] = 0.f;
+        }
+        return;
+    }
+    const long long src = (bh * T + t) * (long long)D;
+    float acc = 0.f;
+    // D/32 consecutive bf16 per lane (2 for D = 64, 4 for D = 128).
+    if (D == 64) {
+        const __nv_bfloat162 a = reinterpret_cast<const __nv_bfloat162*>(o + src)[lane];
+        const __nv_bfloat162 b = reinterpret_cast<const __nv_bfloat162*>(dout + src)[lane];
+        const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+        acc = fa.x * fb.x + fa.y * fb.y;
+        reinterpret_cast<float2*>(dq_acc + src)[lane] = make_float2(0.f, 0.f);
+    } else {
+        const uint2 a = reinterpret_cast<const uint2*>(o + src)[lane];
+        const uint2 b = reinterpret_cast<const uint2*>(dout + src)[lane];
+        const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
+        const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
+        const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.x));
+        const float2 b1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.y));
+        acc = a0.x * b0.x + a0.y * b0.y + a1.x * b1.x + a1.y * b1.y;
+        reinterpret_cast<float4*>(dq_acc + src)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+        delta[row] = acc;
+        lse2[row] = lse[bh * T + t] * 1.4426950408889634f;
+    }
+}
+
+__global__ void attn_dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, long long n8) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n8) return;
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    uint4 r;
+    r.x = pack_bf16x2(a.x, a.y);
+    r.y = pack_bf16x2(a.z, a.w);
+    r.z = pack_bf16x2(b.x, b.y);
+    r.w = pack_bf16x2(b.z, b.w);
+    reinterpret_cast<uint4*>(dq)[i] = r;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const BwdParams p) {
+    using C = BwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    constexpr int kStages = C::kStages;
+    constexpr int kTileBytes = C::kTileBytes;
+    constexpr int kBoxes = D / 64;
+    constexpr uint32_t kTmemCols = 512;
+    constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);    // S^T, dP^T
+    constexpr uint32_t kIdescKxMN = idesc_bf16_f32(128, D, 0, 1);    // dV (A in TMEM), dK
+    constexpr uint32_t kIdescMNxMN = idesc_bf16_f32(128, D, 1, 1);   // dQ
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int bh = blockIdx.x % p.BH;
+    const int kt = blockIdx.x / p.BH;          // key tile 0 sees the most query tiles: launched first
+    const int k0 = kt * kTile;
+    const int qt_lo = kt;
+    const int qt_hi = bwd_last_query_tile(kt, p.n_tiles, p.window);
+    const int n_q = qt_hi - qt_lo + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.bar_kv, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.bar_qdo_full[s], 1);
+            mbar_init(&sm.bar_qdo_empty[s], 1);
+        }
+        mbar_init(&sm.bar_s_full, 1);
+        mbar_init(&sm.bar_dp_full, 1);
+        mbar_init(&sm.bar_p_full, 128);
+        mbar_init(&sm.bar_ds_full, 128);
+        mbar_init(&sm.bar_dv_done, 1);
+        mbar_init(&sm.bar_ds_empty, 1);
+        mbar_init(&sm.bar_dq_full, 1);
+        mbar_init(&sm.bar_dq_empty, 128);
+        mbar_init(&sm.bar_dkdv_full, 1);
+        mbar_init(&sm.bar_drain, 1);
+        sm.abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const AbortCtl ac{&sm.abort_flag, p.timeout_ns};
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_do);
+            mbar_arrive_expect_tx(&sm.bar_kv, 2 * kTileBytes);
+            for (int b = 0; b < kBoxes; ++b) {
+                tma_load_3d(sm.k + b * 16384, &tm_k, &sm.bar_kv, b * 64, k0, bh);
+                tma_load_3d(sm.v + b * 16384, &tm_v, &sm.bar_kv, b * 64, k0, bh);
+            }
+            int it = 0;
+            for (; it < n_q; ++it) {
+                const int s = it % kStages;
+                const int n = it / kStages;
+                if (n > 0 && !mbar_wait(&sm.bar_qdo_empty[s], (n - 1) & 1, ac)) break;
+                const int q0 = (qt_lo + it) * kTile;
+                mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + 2 * kTile * 4);
+                for (int b = 0; b < kBoxes; ++b) {
+                    tma_load_3d(sm.q[s] + b * 16384, &tm_q, &sm.bar_qdo_full[s], b * 64, q0, bh);
+                    tma_load_3d(sm.dout[s] + b * 16384, &tm_do, &sm.bar_qdo_full[s], b * 64, q0, bh);
+                }
+                const size_t roff = (size_t)bh * p.T_pad + q0;
+                bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
+                bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_qdo_full[s]);
+            }
+            if (sm.abort_flag) {
+                mbar_wait_drain(&sm.bar_kv, 0, p.timeout_ns);
+                for (int r = (it > kStages ? it - kStages : 0); r < it; ++r)
+                    mbar_wait_drain(&sm.bar_qdo_full[r % kStages], (r / kStages) & 1, p.timeout_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t k_addr = smem_u32(sm.k);
+            const uint32_t v_addr = smem_u32(sm.v);
+            const uint32_t ds_addr = smem_u32(sm.ds);
+            bool ok = mbar_wait(&sm.bar_kv, 0, ac);
+            for (int it = 0; ok && it < n_q; ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                const uint32_t q_addr = smem_u32(sm.q[s]);
+                const uint32_t do_addr = smem_u32(sm.dout[s]);
+                if (!mbar_wait(&sm.bar_qdo_full[s], ph, ac)) break;
+                if (it > 0) {
+                    // S^T columns: the previous dV MMA read P^T from them (and, for D = 128, the
+                    // previous dQ was accumulated there and must have been read out).
+                    if (!mbar_wait(&sm.bar_dv_done, (it - 1) & 1, ac)) break;
+                    if (C::kDqAliasesS && !mbar_wait(&sm.bar_dq_empty, (it - 1) & 1, ac)) break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_ss(tmem + C::kColS, sw128_desc(k_addr + off, 16, 1024), sw128_desc(q_addr + off, 16, 1024),
+                           kIdescSS, kk > 0);
+                }
+                mma_commit(&sm.bar_s_full);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_ss(tmem + C::kColDP, sw128_desc(v_addr + off, 16, 1024),
+                           sw128_desc(do_addr + off, 16, 1024), kIdescSS, kk > 0);
+                }
+                mma_commit(&sm.bar_dp_full);
+                // dV += P^T dO
+                if (!mbar_wait(&sm.bar_p_full, it & 1, ac)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8, sw128_desc(do_addr + kk * 2048, 16384, 1024),
+                           kIdescKxMN, (it > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&sm.bar_dv_done);
+                // dK += dS^T Q
+                if (!mbar_wait(&sm.bar_ds_full, it & 1, ac)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
+                           sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN, (it > 0 || kk > 0) ? 1u : 0u);
+                }
+                // dQ = dS K (needs the dQ columns free; for D = 128 also the dV MMA done with P^T)
+                if (C::kDqAliasesS) {
+                    if (!mbar_wait(&sm.bar_dv_done, it & 1, ac)) break;
+                } else if (it > 0) {
+                    if (!mbar_wait(&sm.bar_dq_empty, (it - 1) & 1, ac)) break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
+                           sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
+                mma_commit(&sm.bar_dq_full);
+                mma_commit(&sm.bar_qdo_empty[s]);
+                mma_commit(&sm.bar_ds_empty);
+            }
+            mma_commit(&sm.bar_dkdv_full);
+            mma_commit(&sm.bar_drain);
+            mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ P / dS warpgroup (thread = key row)
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const int key = k0 + r;
+        const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
+        const int W = p.window;
+        const float sl2 = p.scale_log2;
+        const float scale = p.scale;
+        const uint32_t ds_row = smem_u32(sm.ds) + r * 128;
+        bool ok = true;
+        for (int it = 0; it < n_q; ++it) {
+            const int s = it % kStages;
+            const uint32_t ph = (it / kStages) & 1;
+            const int qt = qt_lo + it;
+            const int q0 = qt * kTile;
+            if (!warp_wait(&sm.bar_qdo_full[s], ph, ac)) { ok = false; break; }
+            if (!warp_wait(&sm.bar_s_full, it & 1, ac)) { ok = false; break; }
+            if (!warp_wait(&sm.bar_dp_full, it & 1, ac)) { ok = false; break; }
+            if (it > 0 && !warp_wait(&sm.bar_ds_empty, (it - 1) & 1, ac)) { ok = false; break; }
+            tc_fence_after();
+            const bool need_mask = (qt == kt) || (W > 0 && q0 + kTile - 1 >= k0 + W);
+            const float* lse2 = sm.lse2[s];
+            const float* dlt = sm.delta[s];
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t rs[32], rd[32];
+                tmem_ld32(t_lane + C::kColS + c * 32, rs);
+                tmem_ld32(t_lane + C::kColDP + c * 32, rd);
+                tmem_wait_ld();
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int col = c * 32 + e;
+                    float p0 = ex2_approx(__uint_as_float(rs[e]) * sl2 - lse2[col]);
+                    float p1 = ex2_approx(__uint_as_float(rs[e + 1]) * sl2 - lse2[col + 1]);
+                    if (need_mask) {
+                        const int qa = q0 + col;
+                        if (key > qa || (W > 0 && qa >= key + W)) p0 = 0.f;
+                        if (key > qa + 1 || (W > 0 && qa + 1 >= key + W)) p1 = 0.f;
+                    }
+                    const float d0 = p0 * (__uint_as_float(rd[e]) - dlt[col]) * scale;
+                    const float d1 = p1 * (__uint_as_float(rd[e + 1]) - dlt[col + 1]) * scale;
+                    pk[e >> 1] = pack_bf16x2(p0, p1);
+                    dk[e >> 1] = pack_bf16x2(d0, d1);
+                }
+                tmem_st16(t_lane + C::kColS + c * 16, pk);
+                // dS^T row r, queries [32c, 32c + 32): 4 chunks of 16 bytes in half c/2, swizzled by row.
+                const uint32_t half = ds_row + (c >> 1) * 16384;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const uint32_t chunk = ((c & 1) * 4 + t) ^ (r & 7);
+                    st_shared_v4(half + chunk * 16, dk[4 * t], dk[4 * t + 1], dk[4 * t + 2], dk[4 * t + 3]);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.bar_p_full);
+            mbar_arrive(&sm.bar_ds_full);
+        }
+        // ---------------------------------------------------------- dK / dV epilogue
+        if (__all_sync(0xffffffffu, ok) && warp_wait(&sm.bar_dkdv_full, 0, ac)) {
+            tc_fence_after();
+            const bool store = key < p.T;
+            const size_t off = ((size_t)bh * p.T + (store ? key : 0)) * D;
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + off;
+                const uint32_t col0 = which == 0 ? C::kColDV : C::kColDK;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t rr[32];
+                    tmem_ld32(t_lane + col0 + c * 32, rr);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2)
+                        pk[e >> 1] = pack_bf16x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
+                    if (store) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                    }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ dQ writer warpgroup (thread = query row)
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
+        for (int it = 0; it < n_q; ++it) {
+            const int q = (qt_lo + it) * kTile + r;
+            if (!warp_wait(&sm.bar_dq_full, it & 1, ac)) break;
+            tc_fence_after();
+            float* dst = p.dq_acc + ((size_t)bh * p.T + (q < p.T ? q : 0)) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t rr[32];
+                tmem_ld32(t_lane + C::kColDQ + c * 32, rr);
+                tmem_wait_ld();
+                if (q < p.T) {
+#pragma unroll
+                    for (int v4 = 0; v4 < 8; ++v4)
+                        red_add_v4(dst + c * 32 + 4 * v4, __uint_as_float(rr[4 * v4]), __uint_as_float(rr[4 * v4 + 1]),
+                                   __uint_as_float(rr[4 * v4 + 2]), __uint_as_float(rr[4 * v4 + 3]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.bar_dq_empty);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace gpt_attn

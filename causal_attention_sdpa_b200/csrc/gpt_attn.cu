@@ -1,0 +1,304 @@
+// C ABI of the attention library: argument checks, TMA descriptor encoding
+// and kernel launches on the caller's stream.  No allocation, no host sync
+// (except in gpt_attn_check, which exists to sync).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#include <mutex>
+
+#include "attn_bwd.cuh"
+#include "attn_fwd.cuh"
+#include "gpt_attn.h"
+
+extern "C" size_t gpt_attn_bwd_workspace_bytes(int B, int H, int T, int D);
+
+namespace gpt_attn {
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 1000ull * 1000ull * 1000ull;   // 1 s per wait
+
+uint64_t wait_timeout_ns() {
+    static uint64_t v = []() -> uint64_t {
+        const char* s = getenv("GPT_ATTN_WAIT_TIMEOUT_MS");
+        if (s && *s) {
+            const long long ms = atoll(s);
+            if (ms > 0) return (uint64_t)ms * 1000000ull;
+        }
+        return kDefaultTimeoutNs;
+    }();
+    return v;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 [BH, T, D] viewed as a 3-D tensor (D, T, BH); 64-column x 128-row boxes,
+// 128-byte swizzle (matches the UMMA 128B-swizzle canonical layout), zero fill
+// outside the tensor so ragged tails read as zeros.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, int BH, int T, int D) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+int check_shape(int B, int H, int T, int D) {
+    if (B < 1 || H < 1 || T < 1) return GPT_ATTN_ERR_SHAPE;
+    if (D != 64 && D != 128) return GPT_ATTN_ERR_UNSUPPORTED_D;
+    // Every element index must fit in int64, and the TMA coordinates (T, B*H) in int32.
+    const long long bh = (long long)B * H;
+    if (bh > 0x7fffffffLL) return GPT_ATTN_ERR_SHAPE;
+    const long long tp = ((long long)T + 127) / 128 * 128;
+    if (tp > (0x7fffffffffffffffLL / D) / bh) return GPT_ATTN_ERR_SHAPE;
+    if ((tp / 128) * bh > 0x7fffffffLL) return GPT_ATTN_ERR_SHAPE;   // grid size
+    return GPT_ATTN_OK;
+}
+
+template <typename Kern>
+bool set_smem(Kern k, size_t bytes) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+}
+
+template <int D>
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH, int T, float scale,
+               int window, cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    if (!make_tmap_bf16(&mq, q, BH, T, D) || !make_tmap_bf16(&mk, k, BH, T, D) || !make_tmap_bf16(&mv, v, BH, T, D))
+        return GPT_ATTN_ERR_CUDA;
+    FwdParams p;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.T = T;
+    p.BH = BH;
+    p.n_tiles = (T + kTile - 1) / kTile;
+    p.window = window > 0 ? window : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.timeout_ns = wait_timeout_ns();
+    const size_t smem = sizeof(FwdSmem<D>) + 1024;
+    if (!set_smem(attn_fwd_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
+    const unsigned grid = (unsigned)((long long)p.n_tiles * BH);
+    attn_fwd_kernel<D><<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
+}
+
+struct WsLayout {
+    float* dq_acc;
+    float* lse2;
+    float* delta;
+    int n_tiles;
+    int T_pad;
+};
+
+WsLayout ws_layout(void* ws, int BH, int T, int D) {
+    WsLayout w;
+    w.n_tiles = (T + kTile - 1) / kTile;
+    w.T_pad = w.n_tiles * kTile;
+    w.dq_acc = static_cast<float*>(ws);
+    w.lse2 = w.dq_acc + (size_t)BH * T * D;
+    w.delta = w.lse2 + (size_t)BH * w.T_pad;
+    return w;
+}
+
+int launch_bwd_delta(const void* o, const float* lse, const void* dout, int BH, int T, int D, void* ws,
+                     cudaStream_t st) {
+    const WsLayout w = ws_layout(ws, BH, T, D);
+    const long long rows = (long long)BH * w.T_pad;
+    const int wpb = 8;
+    const unsigned grid = (unsigned)((rows + wpb - 1) / wpb);
+    attn_bwd_prep_kernel<<<grid, wpb * 32, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
+                                                    static_cast<const __nv_bfloat16*>(dout), lse, w.lse2, w.delta,
+                                                    w.dq_acc, T, w.T_pad, rows, D);
+    return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
+}
+
+template <int D>
+int launch_bwd_grads(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int BH,
+                     int T, float scale, int window, void* ws, cudaStream_t st) {
+    const WsLayout w = ws_layout(ws, BH, T, D);
+    CUtensorMap mq, mk, mv, mdo;
+    if (!make_tmap_bf16(&mq, q, BH, T, D) || !make_tmap_bf16(&mk, k, BH, T, D) || !make_tmap_bf16(&mv, v, BH, T, D) ||
+        !make_tmap_bf16(&mdo, dout, BH, T, D))
+        return GPT_ATTN_ERR_CUDA;
+    BwdParams p;
+    p.lse2 = w.lse2;
+    p.delta = w.delta;
+    p.dq_acc = w.dq_acc;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.T = T;
+    p.T_pad = w.T_pad;
+    p.BH = BH;
+    p.n_tiles = w.n_tiles;
+    p.window = window > 0 ? window : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.scale = scale;
+    p.timeout_ns = wait_timeout_ns();
+    const size_t smem = sizeof(BwdSmem<D>) + 1024;
+    if (!set_smem(attn_bwd_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
+    const unsigned grid = (unsigned)((long long)w.n_tiles * BH);
+    attn_bwd_kernel<D><<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
+    return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
+}
+
+int launch_dq_convert(void* dq, int BH, int T, int D, void* ws, cudaStream_t st) {
+    const WsLayout w = ws_layout(ws, BH, T, D);
+    const long long n8 = (long long)BH * T * D / 8;
+    const int tpb = 256;
+    const unsigned grid = (unsigned)((n8 + tpb - 1) / tpb);
+    attn_dq_convert_kernel<<<grid, tpb, 0, st>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+    return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
+}
+
+int check_ws(int B, int H, int T, int D, const void* ws, size_t ws_bytes) {
+    if (!ws || ws_bytes < gpt_attn_bwd_workspace_bytes(B, H, T, D)) return GPT_ATTN_ERR_WORKSPACE;
+    return misaligned(ws) ? GPT_ATTN_ERR_ALIGN : GPT_ATTN_OK;
+}
+
+__global__ void debug_wait_kernel(uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);   // nothing ever arrives
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const AbortCtl ac{&abort_flag, timeout_ns};
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, ac);
+    __syncthreads();
+}
+
+}  // namespace
+}  // namespace gpt_attn
+
+using namespace gpt_attn;
+
+extern "C" {
+
+int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T, int D,
+                 float scale, int window, void* stream) {
+    if (!q || !k || !v || !o || !lse) return GPT_ATTN_ERR_NULL;
+    const int sc = check_shape(B, H, T, D);
+    if (sc != GPT_ATTN_OK) return sc;
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse)) return GPT_ATTN_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int BH = B * H;
+    return D == 64 ? launch_fwd<64>(q, k, v, o, lse, BH, T, scale, window, st)
+                   : launch_fwd<128>(q, k, v, o, lse, BH, T, scale, window, st);
+}
+
+size_t gpt_attn_bwd_workspace_bytes(int B, int H, int T, int D) {
+    if (check_shape(B, H, T, D) != GPT_ATTN_OK) return 0;
+    const size_t bh = (size_t)B * H;
+    const size_t t_pad = ((size_t)T + 127) / 128 * 128;
+    return 4 * (bh * T * D + 2 * bh * t_pad);
+}
+
+int gpt_attn_bwd_delta(const void* o, const float* lse, const void* dO, int B, int H, int T, int D,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+    if (!o || !lse || !dO) return GPT_ATTN_ERR_NULL;
+    int sc = check_shape(B, H, T, D);
+    if (sc != GPT_ATTN_OK) return sc;
+    if ((sc = check_ws(B, H, T, D, workspace, workspace_bytes)) != GPT_ATTN_OK) return sc;
+    if (misaligned(o) || misaligned(lse) || misaligned(dO)) return GPT_ATTN_ERR_ALIGN;
+    return launch_bwd_delta(o, lse, dO, B * H, T, D, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int gpt_attn_bwd_grads(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B,
+                       int H, int T, int D, float scale, int window, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+    if (!q || !k || !v || !dO || !dk || !dv) return GPT_ATTN_ERR_NULL;
+    int sc = check_shape(B, H, T, D);
+    if (sc != GPT_ATTN_OK) return sc;
+    if ((sc = check_ws(B, H, T, D, workspace, workspace_bytes)) != GPT_ATTN_OK) return sc;
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(dO) || misaligned(dk) || misaligned(dv))
+        return GPT_ATTN_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return D == 64 ? launch_bwd_grads<64>(q, k, v, dO, dk, dv, B * H, T, scale, window, workspace, st)
+                   : launch_bwd_grads<128>(q, k, v, dO, dk, dv, B * H, T, scale, window, workspace, st);
+}
+
+int gpt_attn_bwd_dq_convert(void* dq, int B, int H, int T, int D, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+    if (!dq) return GPT_ATTN_ERR_NULL;
+    int sc = check_shape(B, H, T, D);
+    if (sc != GPT_ATTN_OK) return sc;
+    if ((sc = check_ws(B, H, T, D, workspace, workspace_bytes)) != GPT_ATTN_OK) return sc;
+    if (misaligned(dq)) return GPT_ATTN_ERR_ALIGN;
+    return launch_dq_convert(dq, B * H, T, D, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                 void* dq, void* dk, void* dv, int B, int H, int T, int D, float scale, int window, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return GPT_ATTN_ERR_NULL;
+    int sc = check_shape(B, H, T, D);
+    if (sc != GPT_ATTN_OK) return sc;
+    if ((sc = check_ws(B, H, T, D, workspace, workspace_bytes)) != GPT_ATTN_OK) return sc;
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse) || misaligned(dO) ||
+        misaligned(dq) || misaligned(dk) || misaligned(dv))
+        return GPT_ATTN_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int BH = B * H;
+    if ((sc = launch_bwd_delta(o, lse, dO, BH, T, D, workspace, st)) != GPT_ATTN_OK) return sc;
+    sc = D == 64 ? launch_bwd_grads<64>(q, k, v, dO, dk, dv, BH, T, scale, window, workspace, st)
+                 : launch_bwd_grads<128>(q, k, v, dO, dk, dv, BH, T, scale, window, workspace, st);
+    if (sc != GPT_ATTN_OK) return sc;
+    return launch_dq_convert(dq, BH, T, D, workspace, st);
+}
+
+int gpt_attn_check(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GPT_ATTN_ERR_CUDA;
+    int st = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&st, gpt_attn::g_status, sizeof(int)) != cudaSuccess) return GPT_ATTN_ERR_CUDA;
+    if (cudaMemcpyToSymbol(gpt_attn::g_status, &zero, sizeof(int)) != cudaSuccess) return GPT_ATTN_ERR_CUDA;
+    if (cudaPeekAtLastError() != cudaSuccess) return GPT_ATTN_ERR_CUDA;
+    return st;
+}
+
+const char* gpt_attn_status_string(int status) {
+    switch (status) {
+        case GPT_ATTN_OK: return "ok";
+        case GPT_ATTN_ERR_NULL: return "null pointer argument";
+        case GPT_ATTN_ERR_SHAPE: return "invalid shape (B, H, T must be >= 1; sizes must fit int64)";
+        case GPT_ATTN_ERR_UNSUPPORTED_D: return "unsupported head dimension (D must be 64 or 128)";
+        case GPT_ATTN_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case GPT_ATTN_ERR_CUDA: return "CUDA error";
+        case GPT_ATTN_ERR_TIMEOUT: return "device-side wait timed out";
+        case GPT_ATTN_ERR_WORKSPACE: return "backward workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+int gpt_attn_debug_wait_timeout(int timeout_us, void* stream) {
+    if (timeout_us < 1 || timeout_us > 10 * 1000 * 1000) return GPT_ATTN_ERR_SHAPE;
+    gpt_attn::debug_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((uint64_t)timeout_us * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,140 @@
+/*
+ * gpt_attn -- causal multi-head scaled-dot-product attention for NVIDIA B200
+ * (sm_100a), forward and backward, behind a plain C ABI.
+ *
+ * The operation ("NanoGPT Speedrun baseline", section "El Mecanismo de
+ * Atencion"): for every batch b and head h (heads are an extra batch
+ * dimension, as in the GPT-2 lecture's attention module),
+ *
+ *     O = softmax(scale * Q K^T) V,   with key j blocked for query i when j > i
+ *
+ * (the boolean triu(diagonal=1) mask of "Un GPT desde cero + nanoGPT",
+ * Laboratorio L2.1, True = blocked; blocked scores are -inf before the
+ * softmax, so each row renormalises over its visible keys).  With a window
+ * W >= 1, key j is visible to query i iff i - W < j <= i (the long/short
+ * sliding-window attention of the modded-nanogpt README's technique list).
+ * The backward pass is the exact gradient of sum(O * dO).
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors Q, K, V, O, dO, dQ, dK, dV are bf16, contiguous [B, H, T, D]
+ *     (row-major, D fastest), in device memory owned by the caller.
+ *   - lse is fp32 [B, H, T]: lse[i] = ln sum_{visible j} exp(scale * q_i . k_j),
+ *     the natural-log row log-sum-exp.  Written by the forward pass, read by
+ *     the backward pass.
+ *   - D must be 64 or 128.  T >= 1, B >= 1, H >= 1; B*H*T*D must fit in int64.
+ *   - Every device pointer must be 16-byte aligned (the TMA rule).
+ *   - window <= 0 means plain causal; window >= T is the same as causal.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     only enqueue work: there is no host synchronisation and no allocation.
+ *   - Errors are returned as gpt_attn_status codes; no exceptions, no abort.
+ *     After an error the outputs are unspecified.  Kernels never hang: every
+ *     wait inside them is bounded, and a wait that runs out records
+ *     GPT_ATTN_ERR_TIMEOUT in a per-device status word read by gpt_attn_check.
+ */
+#ifndef GPT_ATTN_H
+#define GPT_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GPT_ATTN_OK = 0,
+    GPT_ATTN_ERR_NULL = 1,            /* a required pointer is NULL */
+    GPT_ATTN_ERR_SHAPE = 2,           /* B, H or T < 1, or B*H*T*D overflows */
+    GPT_ATTN_ERR_UNSUPPORTED_D = 3,   /* D is not 64 or 128 */
+    GPT_ATTN_ERR_ALIGN = 4,           /* a pointer is not 16-byte aligned */
+    GPT_ATTN_ERR_CUDA = 5,            /* a CUDA call or kernel launch failed */
+    GPT_ATTN_ERR_TIMEOUT = 6,         /* a device-side bounded wait ran out */
+    GPT_ATTN_ERR_WORKSPACE = 7        /* backward workspace missing or too small */
+} gpt_attn_status;
+
+/*
+ * Forward pass.  Computes O and lse as defined above.
+ *   q, k, v : const bf16 [B, H, T, D], device.
+ *   o       : bf16 [B, H, T, D], device, written.
+ *   lse     : fp32 [B, H, T], device, written.
+ *   scale   : multiplier of the scores; 1/sqrt(D) gives the softmax(QK^T/sqrt(d_k))
+ *             of the definition (d_k read as the head dimension).
+ *   window  : <= 0 causal; >= 1 sliding window of that many keys (diagonal included).
+ * Returns GPT_ATTN_OK or an error code.  Asynchronous on `stream`.
+ */
+int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int T, int D, float scale, int window, void* stream);
+
+/*
+ * Bytes of device workspace gpt_attn_bwd needs for this shape: an fp32 dQ
+ * accumulator [B, H, T, D] plus two fp32 row vectors per head padded to a
+ * multiple of 128 rows (the log2-scaled lse and Delta_i = dO_i . O_i).
+ * Returns 0 for shapes gpt_attn_bwd would reject.
+ */
+size_t gpt_attn_bwd_workspace_bytes(int B, int H, int T, int D);
+
+/*
+ * Backward pass of L = sum(O * dO).
+ *   q, k, v, o, dO : const bf16 [B, H, T, D], device (o and lse from gpt_attn_fwd
+ *                    with the same q, k, v, scale and window).
+ *   lse            : const fp32 [B, H, T], device.
+ *   dq, dk, dv     : bf16 [B, H, T, D], device, written.
+ *   workspace      : device buffer of at least gpt_attn_bwd_workspace_bytes(B,H,T,D)
+ *                    bytes, 16-byte aligned, owned by the caller; its contents on
+ *                    entry are ignored and on return are unspecified.
+ * The dQ accumulation uses fp32 atomics, so dQ may differ between runs in the
+ * last bits (summation order); dK, dV and the forward pass are deterministic.
+ * Returns GPT_ATTN_OK or an error code.  Asynchronous on `stream`.
+ */
+int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                 const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                 int B, int H, int T, int D, float scale, int window,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The three stages gpt_attn_bwd runs, in this order, exposed so callers can
+ * schedule or time them separately.  Same arguments, layouts, ownership and
+ * error codes as gpt_attn_bwd; the workspace must be the same buffer for all
+ * three calls of one backward pass.
+ *
+ * gpt_attn_bwd_delta: Delta_i = dO_i . O_i and the log2-scaled lse into the
+ *   workspace rows, and zeroes the workspace's fp32 dQ accumulator.
+ *   Memory-bound.
+ * gpt_attn_bwd_grads: the tensor-core pass over (batch*head, 128-key tile):
+ *   writes dK and dV, and adds every dQ contribution into the fp32
+ *   accumulator.
+ * gpt_attn_bwd_dq_convert: dQ = bf16(accumulator).
+ */
+int gpt_attn_bwd_delta(const void* o, const float* lse, const void* dO, int B, int H, int T, int D,
+                       void* workspace, size_t workspace_bytes, void* stream);
+int gpt_attn_bwd_grads(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                       int B, int H, int T, int D, float scale, int window,
+                       void* workspace, size_t workspace_bytes, void* stream);
+int gpt_attn_bwd_dq_convert(void* dq, int B, int H, int T, int D,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's status
+ * word: GPT_ATTN_OK, or GPT_ATTN_ERR_TIMEOUT if a kernel's bounded wait ran
+ * out since the last check, or GPT_ATTN_ERR_CUDA if a CUDA error is pending.
+ * Blocking: keep it out of timed regions.
+ */
+int gpt_attn_check(void* stream);
+
+/* A static, human-readable name for a status code (never NULL). */
+const char* gpt_attn_status_string(int status);
+
+/*
+ * Diagnostic: launches one small kernel that waits on a shared-memory
+ * barrier nothing ever arrives at, with a bound of `timeout_us` microseconds.
+ * The wait runs out, the kernel records GPT_ATTN_ERR_TIMEOUT in the status
+ * word and returns normally, leaving the context usable.  It exists so tests
+ * can show that the bounded waits end instead of hanging; no attention
+ * kernel is involved.  Asynchronous on `stream`.
+ */
+int gpt_attn_debug_wait_timeout(int timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPT_ATTN_H */

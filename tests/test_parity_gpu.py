@@ -1,0 +1,172 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle on
+the same seeded bf16 inputs.
+
+Tolerances (fixed for this path): max |dO| <= 2e-2 on O, <= 5e-2 on dQ/dK/dV,
+relative Frobenius error <= 1e-2 on each, and max |d lse| <= 1e-3.
+
+The five workloads run at full size on the GPU, in the launch configuration
+the benchmark times; the oracle checks every element of every head for the
+four T <= 1024 workloads and a spread of 6 sampled heads (first and last
+included) for the 8192-token sliding-window one.  Small odd shapes cover ragged tails, tiny T,
+windows and both head dimensions over all heads.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from workloads import WORKLOADS, make_inputs, sample_heads
+
+pytestmark = pytest.mark.gpu
+
+TOL_O, TOL_GRAD, TOL_FRO, TOL_LSE = 2e-2, 5e-2, 1e-2, 1e-3
+
+
+@pytest.fixture(scope="module")
+def ga():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import causal_attention_sdpa_b200 as m
+    from causal_attention_sdpa_b200 import build
+    build.build()
+    m.lib()
+    return m
+
+
+def run_gpu(ga, q, k, v, do, scale, window):
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = ga.gpt_attn_fwd(qd, kd, vd, scale=scale, window=window)
+    dq, dk, dv = ga.gpt_attn_bwd(qd, kd, vd, o, lse, dod, scale=scale, window=window)
+    assert ga.gpt_attn_check() == ga.GPT_ATTN_OK
+    return {n: t.float().cpu() for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+
+
+def run_oracle(q, k, v, do, scale, window, heads=None):
+    if heads is not None:
+        sel = lambda t: torch.stack([t[b, h] for b, h in heads])
+        q, k, v, do = sel(q), sel(k), sel(v), sel(do)
+    o, lse = oracle.attn_fwd(q, k, v, scale, window)
+    dq, dk, dv, _ = oracle.attn_bwd(q, k, v, do, scale, window)
+    return {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+
+
+def compare(got, ref, heads=None, label=""):
+    report = {}
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        g = got[name]
+        if heads is not None:
+            g = torch.stack([g[b, h] for b, h in heads])
+        g = g.double().numpy()
+        r = np.asarray(ref[name], dtype=np.float64).reshape(g.shape)
+        assert np.isfinite(g).all(), f"{label} {name}: non-finite values"
+        d = np.abs(g - r)
+        max_abs = float(d.max()) if d.size else 0.0
+        fro = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30))
+        report[name] = (max_abs, fro)
+        if name == "lse":
+            assert max_abs <= TOL_LSE, f"{label} lse: max |err| {max_abs:.3e}"
+        else:
+            tol = TOL_O if name == "o" else TOL_GRAD
+            assert max_abs <= tol, f"{label} {name}: max |err| {max_abs:.3e} > {tol}"
+            assert fro <= TOL_FRO, f"{label} {name}: rel Frobenius {fro:.3e} > {TOL_FRO}"
+    return report
+
+
+@pytest.mark.parametrize("w", WORKLOADS, ids=[f"cfg{w.index}" for w in WORKLOADS])
+def test_workload_parity(ga, w):
+    q, k, v, do = workloads.workload_inputs(w)
+    got = run_gpu(ga, q, k, v, do, w.scale, w.window)
+    # every head of every tensor, except the 8192-token workload, where the fp64 oracle
+    # checks a spread of 6 of its 24 heads (first and last included)
+    heads = sample_heads(w.B, w.H, 6, seed=w.index) if w.T > 4096 else None
+    ref = run_oracle(q, k, v, do, w.scale, w.window, heads)
+    compare(got, ref, heads, label=f"cfg{w.index}")
+
+
+ODD = [
+    # (B, H, T, D, window, scale)
+    (1, 1, 1, 64, 0, 0.125),
+    (1, 2, 2, 64, 0, 0.125),
+    (2, 1, 17, 64, 0, 0.125),
+    (1, 2, 127, 64, 0, 0.125),
+    (1, 2, 129, 64, 0, 0.125),
+    (1, 1, 1000, 64, 0, 0.125),
+    (1, 2, 300, 64, 1, 0.125),
+    (1, 2, 1000, 64, 128, 0.125),
+    (1, 1, 1000, 64, 1000, 0.125),
+    (1, 1, 700, 64, 200, 0.3),
+    (1, 1, 1, 128, 0, 0.12),
+    (1, 2, 17, 128, 0, 0.12),
+    (1, 2, 129, 128, 0, 0.12),
+    (1, 1, 1000, 128, 128, 0.12),
+    (1, 1, 777, 128, 333, 0.12),
+    (1, 1, 513, 128, 0, 0.088),
+]
+
+
+@pytest.mark.parametrize("B,H,T,D,W,s", ODD, ids=[f"B{c[0]}H{c[1]}T{c[2]}D{c[3]}W{c[4]}" for c in ODD])
+def test_odd_shapes(ga, B, H, T, D, W, s):
+    q, k, v, do = make_inputs(B, H, T, D, seed=T * 7 + D + W)
+    got = run_gpu(ga, q, k, v, do, s, W)
+    ref = run_oracle(q, k, v, do, s, W)
+    compare(got, ref, label=f"B{B}H{H}T{T}D{D}W{W}")
+
+
+def test_qk_normed_small(ga):
+    q, k, v, do = make_inputs(2, 2, 640, 128, seed=99, qk_norm=True)
+    got = run_gpu(ga, q, k, v, do, 0.12, 256)
+    compare(got, run_oracle(q, k, v, do, 0.12, 256), label="qknorm")
+
+
+def test_outputs_fully_written(ga):
+    """Poison every output with NaN first: every element must be overwritten."""
+    B, H, T, D = 2, 3, 333, 64
+    q, k, v, do = (t.cuda() for t in make_inputs(B, H, T, D, seed=5))
+    nan = float("nan")
+    o = torch.full_like(q, nan)
+    lse = torch.full((B, H, T), nan, device="cuda")
+    ga.gpt_attn_fwd(q, k, v, o=o, lse=lse)
+    dq, dk, dv = (torch.full_like(q, nan) for _ in range(3))
+    ws = torch.full((ga.gpt_attn_bwd_workspace_bytes(B, H, T, D) // 4,), nan, device="cuda")
+    ga.gpt_attn_bwd(q, k, v, o, lse, do, dq=dq, dk=dk, dv=dv, workspace=ws)
+    assert ga.gpt_attn_check() == ga.GPT_ATTN_OK
+    for t in (o, lse, dq, dk, dv):
+        assert torch.isfinite(t).all()
+
+
+def test_forward_is_deterministic(ga):
+    q, k, v, do = (t.cuda() for t in make_inputs(2, 4, 1024, 64, seed=6))
+    o1, l1 = ga.gpt_attn_fwd(q, k, v)
+    o2, l2 = ga.gpt_attn_fwd(q, k, v)
+    dq1, dk1, dv1 = ga.gpt_attn_bwd(q, k, v, o1, l1, do)
+    dq2, dk2, dv2 = ga.gpt_attn_bwd(q, k, v, o1, l1, do)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    # dQ sums in fp32 with atomics: equal up to summation order, then bf16 rounding
+    assert (dq1.float() - dq2.float()).abs().max().item() <= 2 ** -6 * dq1.float().abs().max().item()
+
+
+def test_nonzero_stream(ga):
+    s = torch.cuda.Stream()
+    q, k, v, do = (t.cuda() for t in make_inputs(1, 2, 256, 64, seed=7))
+    ref_o, ref_l = ga.gpt_attn_fwd(q, k, v)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        o, l = ga.gpt_attn_fwd(q, k, v, stream=s)
+    s.synchronize()
+    assert torch.equal(o, ref_o) and torch.equal(l, ref_l)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(ga):
+    assert ga.gpt_attn_check() == ga.GPT_ATTN_OK
+    assert ga.gpt_attn_debug_wait_timeout(2000) == ga.GPT_ATTN_OK
+    assert ga.gpt_attn_check() == ga.GPT_ATTN_ERR_TIMEOUT
+    assert ga.gpt_attn_check() == ga.GPT_ATTN_OK   # cleared by the read
+    # the context is still usable
+    q, k, v, do = make_inputs(1, 1, 64, 64, seed=8)
+    got = run_gpu(ga, q, k, v, do, 0.125, 0)
+    compare(got, run_oracle(q, k, v, do, 0.125, 0), label="after-timeout")
