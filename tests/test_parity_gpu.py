@@ -64,14 +64,19 @@ def compare(got, ref, heads=None, label=""):
         assert np.isfinite(g).all(), f"{label} {name}: non-finite values"
         d = np.abs(g - r)
         max_abs = float(d.max()) if d.size else 0.0
-        fro = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30))
+        ref_norm = float(np.linalg.norm(r))
+        fro = float(np.linalg.norm(g - r) / max(ref_norm, 1e-30))
         report[name] = (max_abs, fro)
         if name == "lse":
             assert max_abs <= TOL_LSE, f"{label} lse: max |err| {max_abs:.3e}"
         else:
             tol = TOL_O if name == "o" else TOL_GRAD
             assert max_abs <= tol, f"{label} {name}: max |err| {max_abs:.3e} > {tol}"
-            assert fro <= TOL_FRO, f"{label} {name}: rel Frobenius {fro:.3e} > {TOL_FRO}"
+            # A relative error needs a non-zero reference.  With window 1, or T = 1, every query
+            # sees only itself, so the exact dQ and dK are identically zero (the oracle returns
+            # ~1e-17 rounding); only the absolute bound applies there.
+            if ref_norm > 1e-6 * math.sqrt(r.size):
+                assert fro <= TOL_FRO, f"{label} {name}: rel Frobenius {fro:.3e} > {TOL_FRO}"
     return report
 
 
