@@ -34,7 +34,7 @@ GPT_ATTN_ERR_WORKSPACE = 7
 
 EXPORTED = ("gpt_attn_fwd", "gpt_attn_bwd", "gpt_attn_bwd_workspace_bytes", "gpt_attn_bwd_delta",
             "gpt_attn_bwd_grads", "gpt_attn_bwd_dq_convert", "gpt_attn_check", "gpt_attn_status_string",
-            "gpt_attn_debug_wait_timeout")
+            "gpt_attn_debug_wait_timeout", "gpt_attn_bwd_noalloc")
 
 _lib = None
 
@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.gpt_attn_check.restype = i
         L.gpt_attn_status_string.argtypes = [i]
         L.gpt_attn_status_string.restype = ctypes.c_char_p
+        L.gpt_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+        L.gpt_attn_bwd_noalloc.restype = i
         L.gpt_attn_debug_wait_timeout.argtypes = [i, vp]
         L.gpt_attn_debug_wait_timeout.restype = i
         _lib = L
@@ -145,6 +147,29 @@ def gpt_attn_bwd(q, k, v, o, lse, dO, scale=None, window=0, dq=None, dk=None, dv
                             _stream_handle(stream))
     if rc != GPT_ATTN_OK:
         raise GptAttnError(rc, "gpt_attn_bwd")
+    return dq, dk, dv
+
+
+def gpt_attn_bwd_noalloc(q, k, v, o, lse, dO, scale=None, window=0, dq=None, dk=None, dv=None, stream=None):
+    """gpt_attn_bwd with the library's built-in 32 MiB scratch instead of a workspace argument.
+
+    For callers that must not allocate device memory when the backward pass runs.  Pass
+    dq, dk and dv to keep this wrapper itself allocation-free.  Calls that overlap on the
+    GPU share the scratch and race; the first call on a device should precede any capture.
+    """
+    import torch
+    B, H, T, D = q.shape
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO)):
+        _check_bf16(n, t, q.shape)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    rc = lib().gpt_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk),
+                                    _ptr(dv), B, H, T, D, float(scale), int(window), _stream_handle(stream))
+    if rc != GPT_ATTN_OK:
+        raise GptAttnError(rc, "gpt_attn_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -193,6 +193,36 @@ __global__ void debug_wait_kernel(uint64_t timeout_ns) {
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------------------
+// Built-in scratch for gpt_attn_bwd_noalloc.  A file-scope device array is
+// created when the library's module is loaded on a device and lives until the
+// process exits, so the entry point below never allocates.  In host code the
+// name g_noalloc_scratch is only a host-side shadow symbol, not a device
+// address: the device address is looked up with cudaGetSymbolAddress, once
+// per device, with that device current.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on the
+// first call per device), or nullptr on a CUDA error.
+void* noalloc_scratch_current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_scratch_addr[dev] = ptr;
+    }
+    return g_scratch_addr[dev];
+}
+}  // namespace
 }  // namespace gpt_attn
 
 using namespace gpt_attn;
@@ -293,6 +323,22 @@ const char* gpt_attn_status_string(int status) {
         case GPT_ATTN_ERR_WORKSPACE: return "backward workspace missing or too small";
         default: return "unknown status";
     }
+}
+
+int gpt_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv, int B, int H, int T, int D, float scale,
+                         int window, void* stream) {
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return GPT_ATTN_ERR_NULL;
+    const int sc = check_shape(B, H, T, D);
+    if (sc != GPT_ATTN_OK) return sc;
+    const size_t need = gpt_attn_bwd_workspace_bytes(B, H, T, D);
+    if (need > kNoAllocScratchBytes) return GPT_ATTN_ERR_WORKSPACE;
+    void* ws = noalloc_scratch_current_device();
+    if (!ws) return GPT_ATTN_ERR_CUDA;
+    // The scratch keeps whatever the previous call left; the gpt_attn_bwd stages
+    // rewrite every byte they read (dQ accumulator zeroed, row vectors written
+    // including padding), so nothing else needs clearing here.
+    return gpt_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, window, ws, need, stream);
 }
 
 int gpt_attn_debug_wait_timeout(int timeout_us, void* stream) {

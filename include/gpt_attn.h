@@ -113,6 +113,33 @@ int gpt_attn_bwd_dq_convert(void* dq, int B, int H, int T, int D,
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * gpt_attn_bwd without a caller-supplied workspace, for callers that cannot
+ * allocate device memory at the point where they run the backward pass: for
+ * example code running inside an engine's enqueue step or a host callback,
+ * where cudaMalloc is not allowed, or a process whose device memory is owned
+ * entirely by a pooling allocator that must not be bypassed.  (The pages
+ * describe no such entry point; this is a library convenience.)
+ *
+ * The workspace is a fixed array inside the library, 32 MiB (33554432 bytes)
+ * per GPU, created when the library is loaded on that GPU and kept until the
+ * process exits.  Shapes whose gpt_attn_bwd_workspace_bytes(B,H,T,D) exceeds
+ * 32 MiB are rejected with GPT_ATTN_ERR_WORKSPACE (for example B=8, H=12,
+ * T=1024, D=64 fits; B=64, H=12, T=1024, D=64 does not).  Nothing is
+ * allocated or freed: no cudaMalloc, no cudaFree.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls on a device share the one array, so
+ * calls whose work overlaps on the GPU (different streams, or several host
+ * threads) race with each other: serialise them, e.g. on one stream.
+ * Arguments, layouts, results and the other error codes are those of
+ * gpt_attn_bwd.  Asynchronous on `stream`.
+ */
+int gpt_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                         int B, int H, int T, int D, float scale, int window, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status
  * word: GPT_ATTN_OK, or GPT_ATTN_ERR_TIMEOUT if a kernel's bounded wait ran
  * out since the last check, or GPT_ATTN_ERR_CUDA if a CUDA error is pending.
