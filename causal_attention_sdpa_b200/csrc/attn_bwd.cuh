@@ -172,8 +172,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bh = blockIdx.x % p.BH;
-    const int kt = blockIdx.x / p.BH;          // key tile 0 sees the most query tiles: launched first
+    // Blocks of one head are adjacent in launch order (its Q, dO and dQ rows stay in
+    // L2 across its key tiles); key tile 0 sees the most query tiles and launches first.
+    const int bh = blockIdx.x / p.n_tiles;
+    const int kt = blockIdx.x % p.n_tiles;
     const int k0 = kt * kTile;
     const int qt_lo = kt;
     const int qt_hi = bwd_last_query_tile(kt, p.n_tiles, p.window);
@@ -334,8 +336,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (it > 0 && !warp_wait(&sm.bar_ds_empty, (it - 1) & 1, ac)) { ok = false; break; }
             tc_fence_after();
             const bool need_mask = (qt == kt) || (W > 0 && q0 + kTile - 1 >= k0 + W);
-            const float* lse2 = sm.lse2[s];
-            const float* dlt = sm.delta[s];
+            const uint32_t lse2_a = smem_u32(sm.lse2[s]);
+            const uint32_t dlt_a = smem_u32(sm.delta[s]);
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t rs[32], rd[32];
@@ -346,15 +348,17 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const int col = c * 32 + e;
-                    float p0 = ex2_approx(__uint_as_float(rs[e]) * sl2 - lse2[col]);
-                    float p1 = ex2_approx(__uint_as_float(rs[e + 1]) * sl2 - lse2[col + 1]);
+                    const float2 ls = lds_f32x2(lse2_a + col * 4);
+                    const float2 dl = lds_f32x2(dlt_a + col * 4);
+                    float p0 = ex2_approx(__uint_as_float(rs[e]) * sl2 - ls.x);
+                    float p1 = ex2_approx(__uint_as_float(rs[e + 1]) * sl2 - ls.y);
                     if (need_mask) {
                         const int qa = q0 + col;
                         if (key > qa || (W > 0 && qa >= key + W)) p0 = 0.f;
                         if (key > qa + 1 || (W > 0 && qa + 1 >= key + W)) p1 = 0.f;
                     }
-                    const float d0 = p0 * (__uint_as_float(rd[e]) - dlt[col]) * scale;
-                    const float d1 = p1 * (__uint_as_float(rd[e + 1]) - dlt[col + 1]) * scale;
+                    const float d0 = p0 * (__uint_as_float(rd[e]) - dl.x) * scale;
+                    const float d1 = p1 * (__uint_as_float(rd[e + 1]) - dl.y) * scale;
                     pk[e >> 1] = pack_bf16x2(p0, p1);
                     dk[e >> 1] = pack_bf16x2(d0, d1);
                 }

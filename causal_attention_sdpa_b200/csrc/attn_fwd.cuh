@@ -6,16 +6,28 @@
 // running max m and running sum l, rescaling the old sum by e^(m_old - m_new)
 // when the max grows).  The mapping onto sm_100a is this file's own:
 //
-//   one CTA = one (batch*head, 128-query tile), 6 warps:
-//     warp 0      TMA producer: Q once, then K_j / V_j through a 2-stage ring
-//     warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//     warps 2..5  softmax warpgroup: thread r owns query row r of the tile
-//   TMEM (256 columns): S = Q K_j^T fp32 in columns [0,128); P (bf16 pairs)
-//   is written back over the first 64 of them and fed to the PV MMA straight
-//   from TMEM; the O accumulator lives in columns [128, 128 + D).
+//   one CTA = one (batch*head, 256-query block) = two 128-row Q tiles sharing
+//   every K/V tile it loads; 12 warps:
+//     warp 0       TMA producer: Q0, Q1 once, then K_j / V_j through a ring
+//     warp 1       TMEM allocator and single-thread tcgen05.mma issuer
+//     warps 4..7   softmax warpgroup of Q tile 0 (thread r owns query row r)
+//     warps 8..11  softmax warpgroup of Q tile 1
+//   TMEM (512 columns):
+//     D = 64 : S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O0 [384,448) O1 [448,512)
+//     D = 128: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_t is written over S_t
+//   With separate P columns (D = 64) a softmax warpgroup hands its S columns back as
+//   soon as it has read them into registers, so the MMA warp computes S(j+1) while the
+//   exponentials of S(j) are still running; the issue order per key tile is
+//   S0(j+1) S1(j+1) PV0(j) PV1(j).  With P written over S (D = 128) the order is
+//   PV0(j) S0(j+1) PV1(j) S1(j+1) and each S waits for the PV that read its columns.
 //
-// Tiles of keys entirely after the tile's last query, or entirely before the
-// window of its first query, are never loaded; only the diagonal tile and the
+// The running max is rescaled lazily: O and l are rescaled only when a row's max
+// grows by more than 8 (log2 units) over the max the exponentials use.  Every
+// probability then stays <= 2^8, and since the final O / l and lse use the same
+// reference max the result is unchanged.
+//
+// Key tiles entirely after a Q tile's last query, or entirely before the window
+// of its first query, are never loaded for it; only the diagonal tile and the
 // window-edge tiles evaluate the visibility predicate.
 #pragma once
 
@@ -24,8 +36,8 @@
 namespace gpt_attn {
 
 constexpr int kTile = 128;           // rows per Q tile and per K/V tile
-constexpr int kFwdStages = 2;        // K/V ring depth
-constexpr int kFwdThreads = 192;
+constexpr int kFwdThreads = 384;
+constexpr float kLazyRescale = 8.0f; // log2 units
 
 struct FwdParams {
     __nv_bfloat16* o;
@@ -33,75 +45,108 @@ struct FwdParams {
     int T;
     int BH;
     int n_tiles;          // ceil(T / 128)
+    int n_blocks;         // ceil(n_tiles / 2): 256-query blocks per head
     int window;           // <= 0: causal only
     float scale_log2;     // scale * log2(e)
     uint64_t timeout_ns;
 };
 
 template <int D>
+struct FwdCfg {
+    static constexpr int kStages = (D == 64) ? 3 : 2;
+    static constexpr int kTileBytes = kTile * D * 2;
+    static constexpr bool kSeparateP = (D == 64);
+    static constexpr uint32_t kColS0 = 0, kColS1 = 128;
+    static constexpr uint32_t kColP0 = kSeparateP ? 256u : 0u, kColP1 = kSeparateP ? 320u : 128u;
+    static constexpr uint32_t kColO0 = kSeparateP ? 384u : 256u, kColO1 = kSeparateP ? 448u : 384u;
+};
+
+template <int D>
 struct FwdSmem {
-    static constexpr int kTileBytes = kTile * D * 2;   // one bf16 [128, D] tile
-    alignas(1024) uint8_t q[kTileBytes];
-    alignas(1024) uint8_t k[kFwdStages][kTileBytes];
-    alignas(1024) uint8_t v[kFwdStages][kTileBytes];
+    using C = FwdCfg<D>;
+    alignas(1024) uint8_t q[2][C::kTileBytes];
+    alignas(1024) uint8_t k[C::kStages][C::kTileBytes];
+    alignas(1024) uint8_t v[C::kStages][C::kTileBytes];
     uint64_t bar_q;
-    uint64_t bar_k[kFwdStages];
-    uint64_t bar_v[kFwdStages];
-    uint64_t bar_kv_empty[kFwdStages];
-    uint64_t bar_s_full;
-    uint64_t bar_p_full;
-    uint64_t bar_pv_done;
+    uint64_t bar_k[C::kStages];
+    uint64_t bar_v[C::kStages];
+    uint64_t bar_kv_empty[C::kStages];
+    uint64_t bar_s_full[2];
+    uint64_t bar_s_free[2];
+    uint64_t bar_p_full[2];
+    uint64_t bar_o_done[2];
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort_flag;
 };
 
-// Key range of a query tile: tiles [j_lo, j_hi] hold every visible key.
-__device__ __forceinline__ void fwd_key_range(int q_tile, int window, int& j_lo, int& j_hi) {
-    const int q0 = q_tile * kTile;
-    j_hi = q_tile;
-    j_lo = 0;
+// Key tiles [lo, hi] hold every key visible to some query of Q tile qt.
+__device__ __forceinline__ void fwd_key_range(int qt, int window, int& lo, int& hi) {
+    hi = qt;
+    lo = 0;
     if (window > 0) {
-        const int first = q0 - window + 1;
-        j_lo = first > 0 ? first / kTile : 0;
+        const int first = qt * kTile - window + 1;
+        lo = first > 0 ? first / kTile : 0;
     }
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// (a, b) * s - m on the packed fp32x2 pipe.
+__device__ __forceinline__ void fma2_scale_sub(float& a, float& b, float s, float m) {
+    uint64_t x, sc, mm;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a), "f"(b));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(sc) : "f"(s));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(mm) : "f"(-m));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(x) : "l"(x), "l"(sc), "l"(mm));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(x));
 }
 
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    using C = FwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-    constexpr int kTileBytes = FwdSmem<D>::kTileBytes;
+    constexpr int kStages = C::kStages;
+    constexpr int kTileBytes = C::kTileBytes;
     constexpr int kBoxes = D / 64;                 // 64-column TMA boxes per tile
-    constexpr uint32_t kColS = 0;                  // S / P columns
-    constexpr uint32_t kColO = 128;                // O accumulator columns
-    constexpr uint32_t kTmemCols = 256;
+    constexpr uint32_t kTmemCols = 512;
     constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int bh = blockIdx.x % p.BH;
-    const int q_tile = p.n_tiles - 1 - blockIdx.x / p.BH;   // longest tiles launch first
-    const int q0 = q_tile * kTile;
-    int j_lo, j_hi;
-    fwd_key_range(q_tile, p.window, j_lo, j_hi);
-    const int n_kv = j_hi - j_lo + 1;
+    // Blocks of one head are adjacent in launch order, so a head's K/V tiles are
+    // read from HBM once and then served from L2 to its other query blocks;
+    // within a head the longest blocks launch first.
+    const int bh = blockIdx.x / p.n_blocks;
+    const int qb = p.n_blocks - 1 - blockIdx.x % p.n_blocks;
+    int lo0, hi0, lo1, hi1;
+    fwd_key_range(2 * qb, p.window, lo0, hi0);
+    fwd_key_range(2 * qb + 1, p.window, lo1, hi1);
+    const int j_begin = lo0, j_end = hi1;
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_q, 1);
-        for (int s = 0; s < kFwdStages; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.bar_k[s], 1);
             mbar_init(&sm.bar_v[s], 1);
             mbar_init(&sm.bar_kv_empty[s], 1);
         }
-        mbar_init(&sm.bar_s_full, 1);
-        mbar_init(&sm.bar_p_full, 128);
-        mbar_init(&sm.bar_pv_done, 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&sm.bar_s_full[t], 1);
+            mbar_init(&sm.bar_s_free[t], 128);
+            mbar_init(&sm.bar_p_full[t], 128);
+            mbar_init(&sm.bar_o_done[t], 1);
+        }
         mbar_init(&sm.bar_drain, 1);
         sm.abort_flag = 0;
         fence_barrier_init();
@@ -116,157 +161,209 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const AbortCtl ac{&sm.abort_flag, p.timeout_ns};
-
+    // Launched with 168 registers per thread (384 x 168 = 64512): warpgroup 0
+    // (producer, MMA, two idle warps) drops to 64, the softmax warpgroups take 216.
+    // 128 x 64 + 256 x 216 = 63488 <= 64512.
+    // Each role's code sits under its own setmaxnreg so the compiler allocates it
+    // with that role's budget.
+    if (warp < 4) {
+        regs_dec<64>();
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            mbar_arrive_expect_tx(&sm.bar_q, kTileBytes);
-            for (int b = 0; b < kBoxes; ++b) tma_load_3d(sm.q + b * 16384, &tm_q, &sm.bar_q, b * 64, q0, bh);
+            mbar_arrive_expect_tx(&sm.bar_q, 2 * kTileBytes);
+            for (int t = 0; t < 2; ++t)
+                for (int b = 0; b < kBoxes; ++b)
+                    tma_load_3d(sm.q[t] + b * 16384, &tm_q, &sm.bar_q, b * 64, (2 * qb + t) * kTile, bh);
             int it = 0;
-            for (; it < n_kv; ++it) {
-                const int s = it % kFwdStages;
-                const int n = it / kFwdStages;
+            for (int j = j_begin; j <= j_end; ++j, ++it) {
+                const int s = it % kStages;
+                const int n = it / kStages;
                 if (n > 0 && !mbar_wait(&sm.bar_kv_empty[s], (n - 1) & 1, ac)) break;
-                const int k0 = (j_lo + it) * kTile;
                 mbar_arrive_expect_tx(&sm.bar_k[s], kTileBytes);
                 for (int b = 0; b < kBoxes; ++b)
-                    tma_load_3d(sm.k[s] + b * 16384, &tm_k, &sm.bar_k[s], b * 64, k0, bh);
+                    tma_load_3d(sm.k[s] + b * 16384, &tm_k, &sm.bar_k[s], b * 64, j * kTile, bh);
                 mbar_arrive_expect_tx(&sm.bar_v[s], kTileBytes);
                 for (int b = 0; b < kBoxes; ++b)
-                    tma_load_3d(sm.v[s] + b * 16384, &tm_v, &sm.bar_v[s], b * 64, k0, bh);
+                    tma_load_3d(sm.v[s] + b * 16384, &tm_v, &sm.bar_v[s], b * 64, j * kTile, bh);
             }
             if (sm.abort_flag) {
-                // Let every load already issued land before the CTA exits.
                 mbar_wait_drain(&sm.bar_q, 0, p.timeout_ns);
-                for (int r = (it > kFwdStages ? it - kFwdStages : 0); r < it; ++r) {
-                    const int s = r % kFwdStages, n = r / kFwdStages;
-                    mbar_wait_drain(&sm.bar_k[s], n & 1, p.timeout_ns);
-                    mbar_wait_drain(&sm.bar_v[s], n & 1, p.timeout_ns);
+                for (int r = (it > kStages ? it - kStages : 0); r < it; ++r) {
+                    mbar_wait_drain(&sm.bar_k[r % kStages], (r / kStages) & 1, p.timeout_ns);
+                    mbar_wait_drain(&sm.bar_v[r % kStages], (r / kStages) & 1, p.timeout_ns);
                 }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
+            const uint32_t q_addr0 = smem_u32(sm.q[0]), q_addr1 = smem_u32(sm.q[1]);
             bool ok = mbar_wait(&sm.bar_q, 0, ac);
-            const uint32_t q_addr = smem_u32(sm.q);
-            for (int it = 0; ok && it < n_kv; ++it) {
-                const int s = it % kFwdStages;
-                const uint32_t ph = (it / kFwdStages) & 1;
-                if (!mbar_wait(&sm.bar_k[s], ph, ac)) break;
-                // S shares columns with the P the previous PV MMA reads: wait for it.
-                if (it > 0 && !mbar_wait(&sm.bar_pv_done, (it - 1) & 1, ac)) break;
+            // S_t(j) = Q_t K_j^T into S_t's columns, once those columns are free.
+            auto issue_s = [&](int j, int t) -> bool {
+                const int i = j - (t ? lo1 : lo0);
+                const int it = j - j_begin;
+                const int s = it % kStages;
+                if (!mbar_wait(&sm.bar_k[s], (it / kStages) & 1, ac)) return false;
+                if (i > 0) {
+                    uint64_t* freed = C::kSeparateP ? &sm.bar_s_free[t] : &sm.bar_o_done[t];
+                    if (!mbar_wait(freed, (i - 1) & 1, ac)) return false;
+                }
                 tc_fence_after();
                 const uint32_t k_addr = smem_u32(sm.k[s]);
+                const uint32_t q_addr = t ? q_addr1 : q_addr0;
+                const uint32_t col = t ? C::kColS1 : C::kColS0;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_ss(tmem + kColS, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
+                    mma_ss(tmem + col, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
                            kIdescQK, kk > 0);
                 }
-                mma_commit(&sm.bar_s_full);
-                if (!mbar_wait(&sm.bar_p_full, it & 1, ac)) break;
-                if (!mbar_wait(&sm.bar_v[s], ph, ac)) break;
+                mma_commit(&sm.bar_s_full[t]);
+                return true;
+            };
+            // O_t += P_t V_j once the softmax warpgroup has written P_t(j).
+            auto issue_pv = [&](int j, int t) -> bool {
+                const int i = j - (t ? lo1 : lo0);
+                const int it = j - j_begin;
+                const int s = it % kStages;
+                if (!mbar_wait(&sm.bar_v[s], (it / kStages) & 1, ac)) return false;
+                if (!mbar_wait(&sm.bar_p_full[t], i & 1, ac)) return false;
                 tc_fence_after();
                 const uint32_t v_addr = smem_u32(sm.v[s]);
+                const uint32_t col_o = t ? C::kColO1 : C::kColO0;
+                const uint32_t col_p = t ? C::kColP1 : C::kColP0;
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-                    mma_ts(tmem + kColO, tmem + kColS + kk * 8, sw128_desc(v_addr + kk * 2048, 16384, 1024),
-                           kIdescPV, (it > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ts(tmem + col_o, tmem + col_p + kk * 8, sw128_desc(v_addr + kk * 2048, 16384, 1024),
+                           kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&sm.bar_o_done[t]);
+                return true;
+            };
+            auto active = [&](int j, int t) { return t ? (j >= lo1 && j <= hi1) : (j >= lo0 && j <= hi0); };
+
+            for (int t = 0; ok && t < 2; ++t)
+                if (active(j_begin, t)) ok = issue_s(j_begin, t);
+            for (int j = j_begin; ok && j <= j_end; ++j) {
+                if (C::kSeparateP) {
+                    for (int t = 0; ok && t < 2; ++t)
+                        if (j + 1 <= j_end && active(j + 1, t)) ok = issue_s(j + 1, t);
+                    for (int t = 0; ok && t < 2; ++t)
+                        if (active(j, t)) ok = issue_pv(j, t);
+                } else {
+                    for (int t = 0; ok && t < 2; ++t) {
+                        if (active(j, t)) ok = issue_pv(j, t);
+                        if (ok && j + 1 <= j_end && active(j + 1, t)) ok = issue_s(j + 1, t);
+                    }
                 }
-                mma_commit(&sm.bar_kv_empty[s]);
-                mma_commit(&sm.bar_pv_done);
+                if (ok) mma_commit(&sm.bar_kv_empty[(j - j_begin) % kStages]);
             }
             // Make sure no MMA is still running when TMEM is released.
             mma_commit(&sm.bar_drain);
             mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
         }
+    }
     } else {
-        // ------------------------------------------------------------ softmax warpgroup
-        const int wq = warp & 3;                      // TMEM lane quarter this warp may access
+        regs_inc<216>();
+        // ------------------------------------------------------------ softmax warpgroups
+        const int t = (warp - 4) >> 2;               // Q tile of this warpgroup
+        const int wq = warp & 3;                     // TMEM lane quarter this warp may access
         const int row = wq * 32 + lane;
-        const int i_abs = q0 + row;
+        const int qt = 2 * qb + t;
+        const int i_abs = qt * kTile + row;
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
+        const uint32_t col_s = t ? C::kColS1 : C::kColS0;
+        const uint32_t col_p = t ? C::kColP1 : C::kColP0;
+        const uint32_t col_o = t ? C::kColO1 : C::kColO0;
         const float sl2 = p.scale_log2;
         const int W = p.window;
-        float m = -INFINITY;     // running max, log2 domain
-        float l = 0.f;           // running sum of 2^(x - m)
+        const int lo = t ? lo1 : lo0, hi = t ? hi1 : hi0;
+        float m_used = -INFINITY;    // reference max of the exponentials (log2 units)
+        float l = 0.f;               // running sum of 2^(x - m_used)
         bool ok = true;
-        for (int it = 0; it < n_kv; ++it) {
-            const int k0 = (j_lo + it) * kTile;
-            if (!warp_wait(&sm.bar_s_full, it & 1, ac)) { ok = false; break; }
+        const int n_t = hi - lo + 1;
+        for (int i = 0; i < n_t; ++i) {
+            const int j = lo + i;
+            const int k0 = j * kTile;
+            if (!warp_wait(&sm.bar_s_full[t], i & 1, ac)) { ok = false; break; }
             tc_fence_after();
-            const bool need_mask = (j_lo + it == q_tile) || (W > 0 && k0 <= q0 + kTile - 1 - W);
-            // pass 1: row max of the visible scores in this tile
-            float mx = -INFINITY;
+            float s[128];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t r[32];
-                tmem_ld32(t_lane + kColS + c * 32, r);
-                tmem_wait_ld();
+                tmem_ld32(t_lane + col_s + c * 32, r);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float x = __uint_as_float(r[e]) * sl2;
-                    if (need_mask) {
-                        const int j = k0 + c * 32 + e;
-                        if (j > i_abs || (W > 0 && j <= i_abs - W)) x = -INFINITY;
-                    }
-                    mx = fmaxf(mx, x);
+                for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
+            }
+            tmem_wait_ld();
+            if (C::kSeparateP) {
+                tc_fence_before();
+                mbar_arrive(&sm.bar_s_free[t]);        // S columns may be overwritten now
+            }
+            const bool need_mask = (j == qt) || (W > 0 && k0 <= qt * kTile + kTile - 1 - W);
+            if (need_mask) {
+#pragma unroll
+                for (int e = 0; e < 128; ++e) {
+                    const int jj = k0 + e;
+                    if (jj > i_abs || (W > 0 && jj <= i_abs - W)) s[e] = -INFINITY;
                 }
             }
-            const float m_new = fmaxf(m, mx);
-            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            // tcgen05.ld/st are warp-collective: rescale when any row of the warp needs it
-            // (alpha = 1 for the others).
-            if (it > 0 && __any_sync(0xffffffffu, m_new > m)) {
-                // The previous PV MMA has completed (its commit preceded S's), so O may be rescaled in place.
-                const float alpha = (m_new > m) ? ex2_approx(m - m_use) : 1.f;
+            float mx = fmax3(s[0], s[1], s[2]);
+#pragma unroll
+            for (int e = 3; e < 127; e += 2) mx = fmax3(mx, s[e], s[e + 1]);
+            mx = fmaxf(mx, s[127]);
+            const float m_new = mx * sl2;               // -inf stays -inf (sl2 > 0)
+            const bool need = m_new > m_used + kLazyRescale;
+            if (__any_sync(0xffffffffu, need)) {
+                const float alpha = need ? ex2_approx(m_used - m_new) : 1.f;
+                if (need) m_used = m_new;
                 l *= alpha;
+                if (i > 0) {
+                    // O holds PV up to tile i-1: wait for it, then rescale in place.
+                    if (!warp_wait(&sm.bar_o_done[t], (i - 1) & 1, ac)) { ok = false; break; }
+                    tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(t_lane + kColO + c * 32, r);
-                    tmem_wait_ld();
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(t_lane + col_o + c * 32, r);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                    tmem_st32(t_lane + kColO + c * 32, r);
-                }
-            }
-            m = m_new;
-            // pass 2: probabilities, row sum, bf16 P written over the consumed S columns
-            float rs = 0.f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r[32];
-                tmem_ld32(t_lane + kColS + c * 32, r);
-                tmem_wait_ld();
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float x0 = __uint_as_float(r[e]) * sl2;
-                    float x1 = __uint_as_float(r[e + 1]) * sl2;
-                    if (need_mask) {
-                        const int j = k0 + c * 32 + e;
-                        if (j > i_abs || (W > 0 && j <= i_abs - W)) x0 = -INFINITY;
-                        if (j + 1 > i_abs || (W > 0 && j + 1 <= i_abs - W)) x1 = -INFINITY;
+                        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                        tmem_st32(t_lane + col_o + c * 32, r);
                     }
-                    const float p0 = ex2_approx(x0 - m_use);
-                    const float p1 = ex2_approx(x1 - m_use);
-                    rs += p0 + p1;
-                    pk[e >> 1] = pack_bf16x2(p0, p1);
                 }
-                tmem_st16(t_lane + kColS + c * 16, pk);
             }
-            l += rs;
+            const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
+            float rs0 = 0.f, rs1 = 0.f;
+            uint32_t pk[64];
+#pragma unroll
+            for (int e = 0; e < 128; e += 2) {
+                float a = s[e], b = s[e + 1];
+                fma2_scale_sub(a, b, sl2, m_use);
+                a = ex2_approx(a);
+                b = ex2_approx(b);
+                rs0 += a;
+                rs1 += b;
+                pk[e >> 1] = pack_bf16x2(a, b);
+            }
+            l += rs0 + rs1;
+            // Separate P columns: the previous PV must have finished reading them.
+            if (C::kSeparateP && i > 0) {
+                if (!warp_wait(&sm.bar_o_done[t], (i - 1) & 1, ac)) { ok = false; break; }
+                tc_fence_after();
+            }
+            tmem_st32(t_lane + col_p, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+            tmem_st32(t_lane + col_p + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&sm.bar_p_full);
+            mbar_arrive(&sm.bar_p_full[t]);
         }
         // ---------------------------------------------------------- epilogue
-        if (__all_sync(0xffffffffu, ok) && warp_wait(&sm.bar_pv_done, (n_kv - 1) & 1, ac)) {
+        if (__all_sync(0xffffffffu, ok) && warp_wait(&sm.bar_o_done[t], (n_t - 1) & 1, ac)) {
             tc_fence_after();
             const float inv_l = 1.f / l;
             const bool store = i_abs < p.T;
@@ -274,7 +371,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t r[32];
-                tmem_ld32(t_lane + kColO + c * 32, r);
+                tmem_ld32(t_lane + col_o + c * 32, r);
                 tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
@@ -287,7 +384,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
                 }
             }
-            if (store) p.lse[(size_t)bh * p.T + i_abs] = (m + log2f(l)) * 0.69314718055994531f;
+            if (store) p.lse[(size_t)bh * p.T + i_abs] = (m_used + log2f(l)) * 0.69314718055994531f;
         }
     }
 

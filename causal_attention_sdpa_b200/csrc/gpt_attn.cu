@@ -95,12 +95,13 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.T = T;
     p.BH = BH;
     p.n_tiles = (T + kTile - 1) / kTile;
+    p.n_blocks = (p.n_tiles + 1) / 2;
     p.window = window > 0 ? window : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = wait_timeout_ns();
     const size_t smem = sizeof(FwdSmem<D>) + 1024;
     if (!set_smem(attn_fwd_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
-    const unsigned grid = (unsigned)((long long)p.n_tiles * BH);
+    const unsigned grid = (unsigned)((long long)p.n_blocks * BH);
     attn_fwd_kernel<D><<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
