@@ -220,7 +220,7 @@ def main():
         ga.gpt_attn_bwd_grads(q, k, v, do, dk, dv, ws, scale=w.scale, window=w.window, stream=stream)
         if ev is not None:
             ev[3].record(stream)
-        ga.gpt_attn_bwd_dq_convert(dq, ws, stream=stream)
+        ga.gpt_attn_bwd_dq_convert(dq, ws, scale=w.scale, stream=stream)
         if ev is not None:
             ev[4].record(stream)
 

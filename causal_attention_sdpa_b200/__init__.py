@@ -62,7 +62,7 @@ def lib() -> ctypes.CDLL:
         L.gpt_attn_bwd_delta.restype = i
         L.gpt_attn_bwd_grads.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
         L.gpt_attn_bwd_grads.restype = i
-        L.gpt_attn_bwd_dq_convert.argtypes = [vp, i, i, i, i, vp, sz, vp]
+        L.gpt_attn_bwd_dq_convert.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
         L.gpt_attn_bwd_dq_convert.restype = i
         L.gpt_attn_bwd_workspace_bytes.argtypes = [i, i, i, i]
         L.gpt_attn_bwd_workspace_bytes.restype = sz
@@ -205,11 +205,14 @@ def gpt_attn_bwd_grads(q, k, v, dO, dk, dv, workspace, scale=None, window=0, str
         raise GptAttnError(rc, "gpt_attn_bwd_grads")
 
 
-def gpt_attn_bwd_dq_convert(dq, workspace, stream=None):
-    """Stage 3 of the backward pass (bf16 dQ from the fp32 accumulator)."""
+def gpt_attn_bwd_dq_convert(dq, workspace, scale=None, stream=None):
+    """Stage 3 of the backward pass (bf16 dQ = scale * the fp32 accumulator)."""
     B, H, T, D = dq.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
     ws, nbytes = _ws(workspace, dq)
-    rc = lib().gpt_attn_bwd_dq_convert(_ptr(dq), B, H, T, D, _ptr(ws), nbytes, _stream_handle(stream))
+    rc = lib().gpt_attn_bwd_dq_convert(_ptr(dq), B, H, T, D, float(scale), _ptr(ws), nbytes,
+                                       _stream_handle(stream))
     if rc != GPT_ATTN_OK:
         raise GptAttnError(rc, "gpt_attn_bwd_dq_convert")
 

@@ -7,13 +7,14 @@
 // The pages only call loss.backward(); the decomposition through Delta is an
 // algebraic identity of this gradient, not a different result.
 //
-// Three kernels run in order on the caller's stream:
+// Three stages run in order on the caller's stream:
 //   attn_bwd_prep_kernel   Delta_i = dO_i . O_i and lse*log2(e) into padded
 //                          per-head rows of the workspace; zeroes the fp32 dQ
 //                          accumulator.  HBM-bound.
-//   attn_bwd_kernel<D>     one CTA per (batch*head, 128-key tile); K and V stay
-//                          in shared memory, query tiles stream through a TMA
-//                          ring.  Per query tile, five tcgen05 MMAs:
+//   attn_bwd_kernel (D=64, attn_bwd_d64.cuh) / attn_bwd_serial_kernel (D=128,
+//                          this file): one CTA per (batch*head, 128-key tile);
+//                          K and V stay in shared memory, query tiles stream
+//                          through a TMA ring.  Per query tile, five tcgen05 MMAs:
 //                            S^T  = K Q^T          (TMEM)
 //                            dP^T = V dO^T         (TMEM)
 //                            dV  += P^T dO         (P^T read from TMEM)
@@ -21,9 +22,12 @@
 //                            dQ   = dS K           (same shared tile, MN-major)
 //                          dQ is added into the fp32 accumulator with vector
 //                          red.global.add by a dedicated warpgroup.
-//   attn_dq_convert_kernel fp32 accumulator -> bf16 dQ.
-// The score scale is folded into dS before its bf16 rounding, so dK and dQ
-// need no epilogue scaling.
+//   attn_dq_convert_kernel dQ = bf16(scale * fp32 accumulator).
+// dS is rounded to bf16 unscaled; the score scale is applied once per output
+// element, in the dK epilogue and in the dQ conversion.
+// The serial kernel below runs one query tile at a time through its five MMAs
+// and the P/dS warpgroup; it serves D = 128, whose accumulators fill all 512
+// TMEM columns (dQ reuses the S^T columns).
 #pragma once
 
 #include "attn_fwd.cuh"
@@ -95,66 +99,64 @@ __device__ __forceinline__ int bwd_last_query_tile(int kt, int n_tiles, int wind
     return t < n_tiles - 1 ? (int)t : n_tiles - 1;
 }
 
-__global__ void attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
-                                     const float* __restrict__ lse, float* __restrict__ lse2,
-                                     float* __restrict__ delta, float* __restrict__ dq_acc, int T, int T_pad,
-                                     long long total_rows_pad, int D) {
-    // One warp per padded row.
-    const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= total_rows_pad) return;
-    const long long bh = row / T_pad;
-    const int t = (int)(row - bh * T_pad);
-    if (t >= T) {
-        if (lane == 0) {
-            lse2[row] = INFINITY;
-            delta[row] = 0.f;
-        }
-        return;
-    }
-    const long long src = (bh * T + t) * (long long)D;
+// Delta_i = dO_i . O_i, lse2_i = lse_i * log2(e) for every padded row, and a
+// zeroed fp32 dQ accumulator.  G = D / 8 threads per row, 16-byte accesses.
+// No thread leaves before the group shuffle (every lane of the warp takes part).
+template <int D>
+__global__ void __launch_bounds__(256)
+attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                     const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ delta,
+                     float* __restrict__ dq_acc, int T, int T_pad, long long total_rows_pad) {
+    constexpr int G = D / 8;
+    const long long row = (long long)blockIdx.x * (256 / G) + threadIdx.x / G;
+    const int g = threadIdx.x % G;
+    const bool in_range = row < total_rows_pad;
+    const long long bh = in_range ? row / T_pad : 0;
+    const int t = in_range ? (int)(row - bh * T_pad) : 0;
+    const bool valid = in_range && t < T;
     float acc = 0.f;
-    // D/32 consecutive bf16 per lane (2 for D = 64, 4 for D = 128).
-    if (D == 64) {
-        const __nv_bfloat162 a = reinterpret_cast<const __nv_bfloat162*>(o + src)[lane];
-        const __nv_bfloat162 b = reinterpret_cast<const __nv_bfloat162*>(dout + src)[lane];
-        const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
-        acc = fa.x * fb.x + fa.y * fb.y;
-        reinterpret_cast<float2*>(dq_acc + src)[lane] = make_float2(0.f, 0.f);
-    } else {
-        const uint2 a = reinterpret_cast<const uint2*>(o + src)[lane];
-        const uint2 b = reinterpret_cast<const uint2*>(dout + src)[lane];
-        const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
-        const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
-        const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.x));
-        const float2 b1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.y));
-        acc = a0.x * b0.x + a0.y * b0.y + a1.x * b1.x + a1.y * b1.y;
-        reinterpret_cast<float4*>(dq_acc + src)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+    long long src = 0;
+    if (valid) {
+        src = (bh * T + t) * (long long)D + g * 8;
+        const uint4 a = *reinterpret_cast<const uint4*>(o + src);
+        const uint4 b = *reinterpret_cast<const uint4*>(dout + src);
+        const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
+            const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[e]));
+            acc = fmaf(fa.x, fb.x, acc);
+            acc = fmaf(fa.y, fb.y, acc);
+        }
+        float4* z = reinterpret_cast<float4*>(dq_acc + src);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-        delta[row] = acc;
-        lse2[row] = lse[bh * T + t] * 1.4426950408889634f;
+    for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (in_range && g == 0) {
+        delta[row] = valid ? acc : 0.f;
+        lse2[row] = valid ? lse[bh * T + t] * 1.4426950408889634f : INFINITY;
     }
 }
 
-__global__ void attn_dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, long long n8) {
+__global__ void attn_dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, long long n8,
+                                       float scale) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n8) return;
     const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
     const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
     uint4 r;
-    r.x = pack_bf16x2(a.x, a.y);
-    r.y = pack_bf16x2(a.z, a.w);
-    r.z = pack_bf16x2(b.x, b.y);
-    r.w = pack_bf16x2(b.z, b.w);
+    r.x = pack_bf16x2(a.x * scale, a.y * scale);
+    r.y = pack_bf16x2(a.z * scale, a.w * scale);
+    r.z = pack_bf16x2(b.x * scale, b.y * scale);
+    r.w = pack_bf16x2(b.z * scale, b.w * scale);
     reinterpret_cast<uint4*>(dq)[i] = r;
 }
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
-attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const BwdParams p) {
     using C = BwdCfg<D>;
@@ -322,7 +324,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
         const int W = p.window;
         const float sl2 = p.scale_log2;
-        const float scale = p.scale;
         const uint32_t ds_row = smem_u32(sm.ds) + r * 128;
         bool ok = true;
         for (int it = 0; it < n_q; ++it) {
@@ -357,8 +358,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         if (key > qa || (W > 0 && qa >= key + W)) p0 = 0.f;
                         if (key > qa + 1 || (W > 0 && qa + 1 >= key + W)) p1 = 0.f;
                     }
-                    const float d0 = p0 * (__uint_as_float(rd[e]) - dl.x) * scale;
-                    const float d1 = p1 * (__uint_as_float(rd[e + 1]) - dl.y) * scale;
+                    const float d0 = p0 * (__uint_as_float(rd[e]) - dl.x);
+                    const float d1 = p1 * (__uint_as_float(rd[e + 1]) - dl.y);
                     pk[e >> 1] = pack_bf16x2(p0, p1);
                     dk[e >> 1] = pack_bf16x2(d0, d1);
                 }
@@ -386,6 +387,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int which = 0; which < 2; ++which) {
                 __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + off;
                 const uint32_t col0 = which == 0 ? C::kColDV : C::kColDK;
+                const float mul = which == 0 ? 1.f : p.scale;     // dK = scale * dS^T Q
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t rr[32];
@@ -394,7 +396,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2)
-                        pk[e >> 1] = pack_bf16x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
+                        pk[e >> 1] = pack_bf16x2(__uint_as_float(rr[e]) * mul, __uint_as_float(rr[e + 1]) * mul);
                     if (store) {
                         uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
 #pragma unroll

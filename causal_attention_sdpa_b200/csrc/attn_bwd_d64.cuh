@@ -1,0 +1,353 @@
+// Pipelined backward kernel for head dimension 64 (the GPT-2 shapes).
+//
+// Same gradient and decomposition as attn_bwd.cuh (P, dV = P^T dO, dP, Delta,
+// dS = P (dP - Delta), dK, dQ), same work unit (one CTA per batch*head and
+// 128-key tile, K and V resident in shared memory, query tiles streamed), but
+// the five MMAs of query tile i overlap the P/dS arithmetic of tile i+1:
+//
+//   16 warps:
+//     warp 0        TMA producer (Q, dO, lse, Delta rows through a 3-stage ring)
+//     warp 1        TMEM allocator and single-thread tcgen05.mma issuer
+//     warps 4..7    P/dS warpgroup for query columns [0, 64) of each tile
+//     warps 8..11   P/dS warpgroup for query columns [64, 128)
+//     warps 12..15  dQ warpgroup: reads dQ(i) out of TMEM and adds it into the
+//                   fp32 accumulator with vector reductions; at the end writes
+//                   dK (x scale) and dV
+//   TMEM (512 columns): S^T [0,128)  dP^T [128,256)  P^T bf16 [256,320)
+//                       dV [320,384)  dK [384,448)  dQ [448,512)
+//   Shared memory: K, V; 3 x (Q, dO, lse2, Delta); dS^T bf16 [key][query] x 2.
+//
+// MMA issue order for tile i:  S(i+1) dP(i+1) | dV(i) | dK(i) dQ(i)
+// S(i+1) and dP(i+1) go in as soon as both P/dS warpgroups have copied S(i) and
+// dP(i) into registers, so the tensor pipe computes the next scores while the
+// exponentials of this tile run.
+#pragma once
+
+#include "attn_bwd.cuh"
+
+namespace gpt_attn {
+
+constexpr int kBwd64Threads = 512;
+
+struct Bwd64Cfg {
+    static constexpr int D = 64;
+    static constexpr int kStages = 3;
+    static constexpr int kTileBytes = kTile * D * 2;         // 16 KB
+    static constexpr uint32_t kColS = 0, kColDP = 128, kColP = 256, kColDV = 320, kColDK = 384, kColDQ = 448;
+};
+
+struct Bwd64Smem {
+    using C = Bwd64Cfg;
+    alignas(1024) uint8_t k[C::kTileBytes];
+    alignas(1024) uint8_t v[C::kTileBytes];
+    alignas(1024) uint8_t q[C::kStages][C::kTileBytes];
+    alignas(1024) uint8_t dout[C::kStages][C::kTileBytes];
+    alignas(1024) uint8_t ds[2][kTile * kTile * 2];          // dS^T bf16, two 64-query halves each
+    alignas(16) float lse2[C::kStages][kTile];
+    alignas(16) float delta[C::kStages][kTile];
+    uint64_t bar_kv;
+    uint64_t bar_qdo_full[C::kStages];
+    uint64_t bar_qdo_empty[C::kStages];
+    uint64_t bar_s_full;
+    uint64_t bar_dp_full;
+    uint64_t bar_sdp_free;        // both P/dS warpgroups have S(i), dP(i) in registers
+    uint64_t bar_p_full;          // P^T(i) in TMEM
+    uint64_t bar_dv_done;         // dV(i) MMA finished: P^T columns free
+    uint64_t bar_ds_full[2];      // dS^T(i) in shared buffer i % 2
+    uint64_t bar_ds_empty[2];     // dK(i), dQ(i) finished with buffer i % 2
+    uint64_t bar_dq_full;
+    uint64_t bar_dq_free;         // dQ(i) copied out of TMEM
+    uint64_t bar_dkdv_full;
+    uint64_t bar_drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__global__ void __launch_bounds__(kBwd64Threads, 1)
+attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const BwdParams p) {
+    using C = Bwd64Cfg;
+    constexpr int D = C::D;
+    extern __shared__ uint8_t smem_raw[];
+    Bwd64Smem& sm = *reinterpret_cast<Bwd64Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    constexpr int kStages = C::kStages;
+    constexpr int kTileBytes = C::kTileBytes;
+    constexpr uint32_t kTmemCols = 512;
+    constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);    // S^T = K Q^T, dP^T = V dO^T
+    constexpr uint32_t kIdescKxMN = idesc_bf16_f32(128, D, 0, 1);    // dV (A = P^T in TMEM), dK
+    constexpr uint32_t kIdescMNxMN = idesc_bf16_f32(128, D, 1, 1);   // dQ
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    // Blocks of one head are adjacent in launch order (its Q, dO and dQ rows stay in
+    // L2 across its key tiles); key tile 0 sees the most query tiles and launches first.
+    const int bh = blockIdx.x / p.n_tiles;
+    const int kt = blockIdx.x % p.n_tiles;
+    const int k0 = kt * kTile;
+    const int qt_lo = kt;
+    const int qt_hi = bwd_last_query_tile(kt, p.n_tiles, p.window);
+    const int n_q = qt_hi - qt_lo + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.bar_kv, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.bar_qdo_full[s], 1);
+            mbar_init(&sm.bar_qdo_empty[s], 1);
+        }
+        mbar_init(&sm.bar_s_full, 1);
+        mbar_init(&sm.bar_dp_full, 1);
+        mbar_init(&sm.bar_sdp_free, 256);
+        mbar_init(&sm.bar_p_full, 256);
+        mbar_init(&sm.bar_dv_done, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.bar_ds_full[b], 256);
+            mbar_init(&sm.bar_ds_empty[b], 1);
+        }
+        mbar_init(&sm.bar_dq_full, 1);
+        mbar_init(&sm.bar_dq_free, 128);
+        mbar_init(&sm.bar_dkdv_full, 1);
+        mbar_init(&sm.bar_drain, 1);
+        sm.abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const AbortCtl ac{&sm.abort_flag, p.timeout_ns};
+
+    // Launched with 128 registers per thread (512 x 128 = 65536).  Warpgroup 0
+    // (producer, MMA, 2 idle warps) 56, the two P/dS warpgroups 184, the dQ
+    // warpgroup 88: 128 x (56 + 184 + 184 + 88) = 65536.
+    if (warp < 4) {
+        regs_dec<56>();
+        if (warp == 0 && lane == 0) {
+            // -------------------------------------------------------- producer
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_do);
+            mbar_arrive_expect_tx(&sm.bar_kv, 2 * kTileBytes);
+            tma_load_3d(sm.k, &tm_k, &sm.bar_kv, 0, k0, bh);
+            tma_load_3d(sm.v, &tm_v, &sm.bar_kv, 0, k0, bh);
+            int it = 0;
+            for (; it < n_q; ++it) {
+                const int s = it % kStages;
+                const int n = it / kStages;
+                if (n > 0 && !mbar_wait(&sm.bar_qdo_empty[s], (n - 1) & 1, ac)) break;
+                const int q0 = (qt_lo + it) * kTile;
+                mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + 2 * kTile * 4);
+                tma_load_3d(sm.q[s], &tm_q, &sm.bar_qdo_full[s], 0, q0, bh);
+                tma_load_3d(sm.dout[s], &tm_do, &sm.bar_qdo_full[s], 0, q0, bh);
+                const size_t roff = (size_t)bh * p.T_pad + q0;
+                bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
+                bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_qdo_full[s]);
+            }
+            if (sm.abort_flag) {
+                mbar_wait_drain(&sm.bar_kv, 0, p.timeout_ns);
+                for (int r = (it > kStages ? it - kStages : 0); r < it; ++r)
+                    mbar_wait_drain(&sm.bar_qdo_full[r % kStages], (r / kStages) & 1, p.timeout_ns);
+            }
+        } else if (warp == 1 && lane == 0) {
+            // -------------------------------------------------------- MMA issuer
+            const uint32_t k_addr = smem_u32(sm.k);
+            const uint32_t v_addr = smem_u32(sm.v);
+            auto issue_s_dp = [&](int i) -> bool {
+                const int s = i % kStages;
+                if (!mbar_wait(&sm.bar_qdo_full[s], (i / kStages) & 1, ac)) return false;
+                if (i > 0 && !mbar_wait(&sm.bar_sdp_free, (i - 1) & 1, ac)) return false;
+                tc_fence_after();
+                const uint32_t q_addr = smem_u32(sm.q[s]);
+                const uint32_t do_addr = smem_u32(sm.dout[s]);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + C::kColS, sw128_desc(k_addr + kk * 32, 16, 1024),
+                           sw128_desc(q_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
+                mma_commit(&sm.bar_s_full);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + C::kColDP, sw128_desc(v_addr + kk * 32, 16, 1024),
+                           sw128_desc(do_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
+                mma_commit(&sm.bar_dp_full);
+                return true;
+            };
+            bool ok = mbar_wait(&sm.bar_kv, 0, ac) && issue_s_dp(0);
+            for (int i = 0; ok && i < n_q; ++i) {
+                const int s = i % kStages;
+                const int b = i & 1;
+                if (i + 1 < n_q && !(ok = issue_s_dp(i + 1))) break;
+                const uint32_t q_addr = smem_u32(sm.q[s]);
+                const uint32_t do_addr = smem_u32(sm.dout[s]);
+                const uint32_t ds_addr = smem_u32(sm.ds[b]);
+                // dV += P^T dO
+                if (!(ok = mbar_wait(&sm.bar_p_full, i & 1, ac))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ts(tmem + C::kColDV, tmem + C::kColP + kk * 8, sw128_desc(do_addr + kk * 2048, 16384, 1024),
+                           kIdescKxMN, (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&sm.bar_dv_done);
+                // dK += dS^T Q
+                if (!(ok = mbar_wait(&sm.bar_ds_full[b], (i >> 1) & 1, ac))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
+                           sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN, (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                // dQ = dS K, once the dQ warpgroup has copied out the previous one
+                if (i > 0 && !(ok = mbar_wait(&sm.bar_dq_free, (i - 1) & 1, ac))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
+                           sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
+                mma_commit(&sm.bar_dq_full);
+                mma_commit(&sm.bar_ds_empty[b]);
+                mma_commit(&sm.bar_qdo_empty[s]);
+            }
+            mma_commit(&sm.bar_dkdv_full);
+            mma_commit(&sm.bar_drain);
+            mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
+        }
+    } else if (warp < 12) {
+        regs_inc<184>();
+        // ------------------------------------------------------------ P / dS warpgroups (thread = key row)
+        const int h = (warp - 4) >> 2;              // query-column half of this warpgroup
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const int key = k0 + r;
+        const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
+        const int W = p.window;
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        for (int i = 0; i < n_q; ++i) {
+            const int s = i % kStages;
+            const int b = i & 1;
+            const int qt = qt_lo + i;
+            const int qc0 = qt * kTile + h * 64;       // first query column of this half
+            if (!warp_wait(&sm.bar_qdo_full[s], (i / kStages) & 1, ac)) { ok = false; break; }
+            if (!warp_wait(&sm.bar_s_full, i & 1, ac)) { ok = false; break; }
+            if (!warp_wait(&sm.bar_dp_full, i & 1, ac)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t rs[64], rd[64];
+            tmem_ld32(t_lane + C::kColS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
+            tmem_ld32(t_lane + C::kColS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
+            tmem_ld32(t_lane + C::kColDP + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&rd[0]));
+            tmem_ld32(t_lane + C::kColDP + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rd[32]));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_sdp_free);             // S^T, dP^T columns may be overwritten now
+
+            const bool need_mask = (qt == kt) || (W > 0 && qt * kTile + kTile - 1 >= k0 + W);
+            const uint32_t lse2_a = smem_u32(sm.lse2[s]) + h * 64 * 4;
+            const uint32_t dlt_a = smem_u32(sm.delta[s]) + h * 64 * 4;
+            uint32_t pk[32], dk[32];
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+                const float2 ls = lds_f32x2(lse2_a + e * 4);
+                const float2 dl = lds_f32x2(dlt_a + e * 4);
+                float p0 = ex2_approx(fmaf(__uint_as_float(rs[e]), sl2, -ls.x));
+                float p1 = ex2_approx(fmaf(__uint_as_float(rs[e + 1]), sl2, -ls.y));
+                if (need_mask) {
+                    const int qa = qc0 + e;
+                    if (key > qa || (W > 0 && qa >= key + W)) p0 = 0.f;
+                    if (key > qa + 1 || (W > 0 && qa + 1 >= key + W)) p1 = 0.f;
+                }
+                const float d0 = p0 * (__uint_as_float(rd[e]) - dl.x);
+                const float d1 = p1 * (__uint_as_float(rd[e + 1]) - dl.y);
+                pk[e >> 1] = pack_bf16x2(p0, p1);
+                dk[e >> 1] = pack_bf16x2(d0, d1);
+            }
+            // P^T(i) into TMEM once dV(i-1) has finished reading P^T(i-1)
+            if (i > 0 && !warp_wait(&sm.bar_dv_done, (i - 1) & 1, ac)) { ok = false; break; }
+            tc_fence_after();
+            tmem_st32(t_lane + C::kColP + h * 32, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_p_full);
+            // dS^T(i) into shared buffer b once dK(i-2), dQ(i-2) have finished with it.
+            // Row r of half h holds queries [64h, 64h + 64): 8 chunks of 16 bytes, swizzled by row.
+            if (i >= 2 && !warp_wait(&sm.bar_ds_empty[b], ((i >> 1) - 1) & 1, ac)) { ok = false; break; }
+            const uint32_t row_a = smem_u32(sm.ds[b]) + h * 16384 + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                st_shared_v4(row_a + ((c ^ (r & 7)) << 4), dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.bar_ds_full[b]);
+        }
+        (void)ok;
+    } else {
+        regs_dec<88>();
+        // ------------------------------------------------------------ dQ warpgroup (thread = query / key row)
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
+        bool ok = true;
+        for (int i = 0; i < n_q; ++i) {
+            const int q = (qt_lo + i) * kTile + r;
+            if (!warp_wait(&sm.bar_dq_full, i & 1, ac)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t rr[64];
+            tmem_ld32(t_lane + C::kColDQ, *reinterpret_cast<uint32_t(*)[32]>(&rr[0]));
+            tmem_ld32(t_lane + C::kColDQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&rr[32]));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_dq_free);
+            if (q < p.T) {
+                float* dst = p.dq_acc + ((size_t)bh * p.T + q) * D;
+#pragma unroll
+                for (int v4 = 0; v4 < 16; ++v4)
+                    red_add_v4(dst + 4 * v4, __uint_as_float(rr[4 * v4]), __uint_as_float(rr[4 * v4 + 1]),
+                               __uint_as_float(rr[4 * v4 + 2]), __uint_as_float(rr[4 * v4 + 3]));
+            }
+        }
+        // ---------------------------------------------------------- dK / dV epilogue (thread = key row)
+        if (__all_sync(0xffffffffu, ok) && warp_wait(&sm.bar_dkdv_full, 0, ac)) {
+            tc_fence_after();
+            const int key = k0 + r;
+            const bool store = key < p.T;
+            const size_t off = ((size_t)bh * p.T + (store ? key : 0)) * D;
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + off;
+                const uint32_t col0 = which == 0 ? C::kColDV : C::kColDK;
+                const float mul = which == 0 ? 1.f : p.scale;     // dK = scale * dS^T Q
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t rr[32];
+                    tmem_ld32(t_lane + col0 + c * 32, rr);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2)
+                        pk[e >> 1] = pack_bf16x2(__uint_as_float(rr[e]) * mul, __uint_as_float(rr[e + 1]) * mul);
+                    if (store) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace gpt_attn

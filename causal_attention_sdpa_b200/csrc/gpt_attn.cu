@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "attn_bwd.cuh"
+#include "attn_bwd_d64.cuh"
 #include "attn_fwd.cuh"
 #include "gpt_attn.h"
 
@@ -128,11 +129,14 @@ int launch_bwd_delta(const void* o, const float* lse, const void* dout, int BH, 
                      cudaStream_t st) {
     const WsLayout w = ws_layout(ws, BH, T, D);
     const long long rows = (long long)BH * w.T_pad;
-    const int wpb = 8;
-    const unsigned grid = (unsigned)((rows + wpb - 1) / wpb);
-    attn_bwd_prep_kernel<<<grid, wpb * 32, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
-                                                    static_cast<const __nv_bfloat16*>(dout), lse, w.lse2, w.delta,
-                                                    w.dq_acc, T, w.T_pad, rows, D);
+    const int rows_per_block = 256 / (D / 8);
+    const unsigned grid = (unsigned)((rows + rows_per_block - 1) / rows_per_block);
+    const auto* o16 = static_cast<const __nv_bfloat16*>(o);
+    const auto* do16 = static_cast<const __nv_bfloat16*>(dout);
+    if (D == 64)
+        attn_bwd_prep_kernel<64><<<grid, 256, 0, st>>>(o16, do16, lse, w.lse2, w.delta, w.dq_acc, T, w.T_pad, rows);
+    else
+        attn_bwd_prep_kernel<128><<<grid, 256, 0, st>>>(o16, do16, lse, w.lse2, w.delta, w.dq_acc, T, w.T_pad, rows);
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
@@ -158,19 +162,25 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
     p.scale_log2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.timeout_ns = wait_timeout_ns();
-    const size_t smem = sizeof(BwdSmem<D>) + 1024;
-    if (!set_smem(attn_bwd_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
     const unsigned grid = (unsigned)((long long)w.n_tiles * BH);
-    attn_bwd_kernel<D><<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
+    if constexpr (D == 64) {
+        const size_t smem = sizeof(Bwd64Smem) + 1024;
+        if (!set_smem(attn_bwd_kernel, smem)) return GPT_ATTN_ERR_CUDA;
+        attn_bwd_kernel<<<grid, kBwd64Threads, smem, st>>>(mq, mk, mv, mdo, p);
+    } else {
+        const size_t smem = sizeof(BwdSmem<D>) + 1024;
+        if (!set_smem(attn_bwd_serial_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
+        attn_bwd_serial_kernel<D><<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
+    }
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
-int launch_dq_convert(void* dq, int BH, int T, int D, void* ws, cudaStream_t st) {
+int launch_dq_convert(void* dq, int BH, int T, int D, float scale, void* ws, cudaStream_t st) {
     const WsLayout w = ws_layout(ws, BH, T, D);
     const long long n8 = (long long)BH * T * D / 8;
     const int tpb = 256;
     const unsigned grid = (unsigned)((n8 + tpb - 1) / tpb);
-    attn_dq_convert_kernel<<<grid, tpb, 0, st>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+    attn_dq_convert_kernel<<<grid, tpb, 0, st>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq), n8, scale);
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
@@ -273,14 +283,14 @@ int gpt_attn_bwd_grads(const void* q, const void* k, const void* v, const void* 
                    : launch_bwd_grads<128>(q, k, v, dO, dk, dv, B * H, T, scale, window, workspace, st);
 }
 
-int gpt_attn_bwd_dq_convert(void* dq, int B, int H, int T, int D, void* workspace, size_t workspace_bytes,
-                            void* stream) {
+int gpt_attn_bwd_dq_convert(void* dq, int B, int H, int T, int D, float scale, void* workspace,
+                            size_t workspace_bytes, void* stream) {
     if (!dq) return GPT_ATTN_ERR_NULL;
     int sc = check_shape(B, H, T, D);
     if (sc != GPT_ATTN_OK) return sc;
     if ((sc = check_ws(B, H, T, D, workspace, workspace_bytes)) != GPT_ATTN_OK) return sc;
     if (misaligned(dq)) return GPT_ATTN_ERR_ALIGN;
-    return launch_dq_convert(dq, B * H, T, D, workspace, static_cast<cudaStream_t>(stream));
+    return launch_dq_convert(dq, B * H, T, D, scale, workspace, static_cast<cudaStream_t>(stream));
 }
 
 int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
@@ -299,7 +309,7 @@ int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
     sc = D == 64 ? launch_bwd_grads<64>(q, k, v, dO, dk, dv, BH, T, scale, window, workspace, st)
                  : launch_bwd_grads<128>(q, k, v, dO, dk, dv, BH, T, scale, window, workspace, st);
     if (sc != GPT_ATTN_OK) return sc;
-    return launch_dq_convert(dq, BH, T, D, workspace, st);
+    return launch_dq_convert(dq, BH, T, D, scale, workspace, st);
 }
 
 int gpt_attn_check(void* stream) {

@@ -102,14 +102,15 @@ int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o,
  * gpt_attn_bwd_grads: the tensor-core pass over (batch*head, 128-key tile):
  *   writes dK and dV, and adds every dQ contribution into the fp32
  *   accumulator.
- * gpt_attn_bwd_dq_convert: dQ = bf16(accumulator).
+ * gpt_attn_bwd_dq_convert: dQ = bf16(scale * accumulator) (the accumulator
+ *   holds dS K; `scale` must be the one passed to gpt_attn_bwd_grads).
  */
 int gpt_attn_bwd_delta(const void* o, const float* lse, const void* dO, int B, int H, int T, int D,
                        void* workspace, size_t workspace_bytes, void* stream);
 int gpt_attn_bwd_grads(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
                        int B, int H, int T, int D, float scale, int window,
                        void* workspace, size_t workspace_bytes, void* stream);
-int gpt_attn_bwd_dq_convert(void* dq, int B, int H, int T, int D,
+int gpt_attn_bwd_dq_convert(void* dq, int B, int H, int T, int D, float scale,
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
