@@ -161,8 +161,7 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const BwdParams p) {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
-    BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(smem_align1024(smem_raw));
 
     constexpr int kStages = C::kStages;
     constexpr int kTileBytes = C::kTileBytes;
@@ -337,27 +336,31 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             if (it > 0 && !warp_wait(&sm.bar_ds_empty, (it - 1) & 1, ac)) { ok = false; break; }
             tc_fence_after();
             const bool need_mask = (qt == kt) || (W > 0 && q0 + kTile - 1 >= k0 + W);
-            const uint32_t lse2_a = smem_u32(sm.lse2[s]);
-            const uint32_t dlt_a = smem_u32(sm.delta[s]);
+            const float2* lse2 = reinterpret_cast<const float2*>(sm.lse2[s]);
+            const float2* dlt = reinterpret_cast<const float2*>(sm.delta[s]);
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t rs[32], rd[32];
                 tmem_ld32(t_lane + C::kColS + c * 32, rs);
                 tmem_ld32(t_lane + C::kColDP + c * 32, rd);
                 tmem_wait_ld();
+                if (need_mask) {
+                    // visible query columns of this key: one range, compare + select per element
+                    const int c_lo = key - (q0 + c * 32);
+                    const int c_hi = W > 0 ? key + W - 1 - (q0 + c * 32) : INT_MAX / 2;
+                    const uint32_t span = (uint32_t)(c_hi - c_lo);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        rs[e] = ((uint32_t)(e - c_lo) <= span) ? rs[e] : 0xff800000u;   // -inf: P = 0
+                }
                 uint32_t pk[16], dk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const int col = c * 32 + e;
-                    const float2 ls = lds_f32x2(lse2_a + col * 4);
-                    const float2 dl = lds_f32x2(dlt_a + col * 4);
-                    float p0 = ex2_approx(__uint_as_float(rs[e]) * sl2 - ls.x);
-                    float p1 = ex2_approx(__uint_as_float(rs[e + 1]) * sl2 - ls.y);
-                    if (need_mask) {
-                        const int qa = q0 + col;
-                        if (key > qa || (W > 0 && qa >= key + W)) p0 = 0.f;
-                        if (key > qa + 1 || (W > 0 && qa + 1 >= key + W)) p1 = 0.f;
-                    }
+                    const float2 ls = lse2[col >> 1];
+                    const float2 dl = dlt[col >> 1];
+                    const float p0 = ex2_approx(__uint_as_float(rs[e]) * sl2 - ls.x);
+                    const float p1 = ex2_approx(__uint_as_float(rs[e + 1]) * sl2 - ls.y);
                     const float d0 = p0 * (__uint_as_float(rd[e]) - dl.x);
                     const float d1 = p1 * (__uint_as_float(rd[e + 1]) - dl.y);
                     pk[e >> 1] = pack_bf16x2(p0, p1);

@@ -7,17 +7,19 @@
 //
 //   16 warps:
 //     warp 0        TMA producer (Q, dO, lse, Delta rows through a 3-stage ring)
-//     warp 1        TMEM allocator and single-thread tcgen05.mma issuer
+//     warp 1        TMEM allocator; issues S^T = K Q^T and dP^T = V dO^T
+//     warp 2        issues dV += P^T dO        warp 3   issues dK += dS^T Q
 //     warps 4..7    P/dS warpgroup for query columns [0, 64) of each tile
 //     warps 8..11   P/dS warpgroup for query columns [64, 128)
-//     warps 12..15  dQ warpgroup: reads dQ(i) out of TMEM and adds it into the
-//                   fp32 accumulator with vector reductions; at the end writes
-//                   dK (x scale) and dV
+//     warps 12..15  dQ warpgroup: issues dQ = dS K, reads it out of TMEM and adds
+//                   it into the fp32 accumulator with vector reductions; at the
+//                   end writes dK (x scale) and dV
+//   Each MMA kind has its own issuing warp: one thread cannot issue 128-row
+//   MMAs of N <= 128 fast enough to keep the tensor pipe busy, four can.
 //   TMEM (512 columns): S^T [0,128)  dP^T [128,256)  P^T bf16 [256,320)
 //                       dV [320,384)  dK [384,448)  dQ [448,512)
 //   Shared memory: K, V; 3 x (Q, dO, lse2, Delta); dS^T bf16 [key][query] x 2.
 //
-// MMA issue order for tile i:  S(i+1) dP(i+1) | dV(i) | dK(i) dQ(i)
 // S(i+1) and dP(i+1) go in as soon as both P/dS warpgroups have copied S(i) and
 // dP(i) into registers, so the tensor pipe computes the next scores while the
 // exponentials of this tile run.
@@ -70,7 +72,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     using C = Bwd64Cfg;
     constexpr int D = C::D;
     extern __shared__ uint8_t smem_raw[];
-    Bwd64Smem& sm = *reinterpret_cast<Bwd64Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bwd64Smem& sm = *reinterpret_cast<Bwd64Smem*>(smem_align1024(smem_raw));
 
     constexpr int kStages = C::kStages;
     constexpr int kTileBytes = C::kTileBytes;
@@ -94,7 +96,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(&sm.bar_kv, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.bar_qdo_full[s], 1);
-            mbar_init(&sm.bar_qdo_empty[s], 1);
+            mbar_init(&sm.bar_qdo_empty[s], 2);     // dV warp + dK warp
         }
         mbar_init(&sm.bar_s_full, 1);
         mbar_init(&sm.bar_dp_full, 1);
@@ -103,12 +105,12 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(&sm.bar_dv_done, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.bar_ds_full[b], 256);
-            mbar_init(&sm.bar_ds_empty[b], 1);
+            mbar_init(&sm.bar_ds_empty[b], 2);      // dK warp + dQ issuer
         }
         mbar_init(&sm.bar_dq_full, 1);
         mbar_init(&sm.bar_dq_free, 128);
-        mbar_init(&sm.bar_dkdv_full, 1);
-        mbar_init(&sm.bar_drain, 1);
+        mbar_init(&sm.bar_dkdv_full, 2);            // last dV + last dK
+        mbar_init(&sm.bar_drain, 4);                // the four MMA-issuing threads
         sm.abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -155,68 +157,73 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int r = (it > kStages ? it - kStages : 0); r < it; ++r)
                     mbar_wait_drain(&sm.bar_qdo_full[r % kStages], (r / kStages) & 1, p.timeout_ns);
             }
-        } else if (warp == 1 && lane == 0) {
-            // -------------------------------------------------------- MMA issuer
+        } else if (lane == 0) {
+            // -------------------------------------------------------- MMA issuers
+            // One tcgen05.mma stream per warp (a single issuing thread cannot keep the
+            // tensor pipe busy with N <= 128 MMAs): warp 1 S^T and dP^T, warp 2 dV,
+            // warp 3 dK; dQ is issued by the dQ warpgroup itself.
             const uint32_t k_addr = smem_u32(sm.k);
             const uint32_t v_addr = smem_u32(sm.v);
-            auto issue_s_dp = [&](int i) -> bool {
-                const int s = i % kStages;
-                if (!mbar_wait(&sm.bar_qdo_full[s], (i / kStages) & 1, ac)) return false;
-                if (i > 0 && !mbar_wait(&sm.bar_sdp_free, (i - 1) & 1, ac)) return false;
-                tc_fence_after();
-                const uint32_t q_addr = smem_u32(sm.q[s]);
-                const uint32_t do_addr = smem_u32(sm.dout[s]);
+            bool ok = true;
+            if (warp == 1) {
+                ok = mbar_wait(&sm.bar_kv, 0, ac);
+                for (int i = 0; ok && i < n_q; ++i) {
+                    const int s = i % kStages;
+                    if (!(ok = mbar_wait(&sm.bar_qdo_full[s], (i / kStages) & 1, ac))) break;
+                    if (i > 0 && !(ok = mbar_wait(&sm.bar_sdp_free, (i - 1) & 1, ac))) break;
+                    tc_fence_after();
+                    const uint32_t q_addr = smem_u32(sm.q[s]);
+                    const uint32_t do_addr = smem_u32(sm.dout[s]);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(tmem + C::kColS, sw128_desc(k_addr + kk * 32, 16, 1024),
-                           sw128_desc(q_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
-                mma_commit(&sm.bar_s_full);
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(tmem + C::kColS, sw128_desc(k_addr + kk * 32, 16, 1024),
+                               sw128_desc(q_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
+                    mma_commit(&sm.bar_s_full);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_ss(tmem + C::kColDP, sw128_desc(v_addr + kk * 32, 16, 1024),
-                           sw128_desc(do_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
-                mma_commit(&sm.bar_dp_full);
-                return true;
-            };
-            bool ok = mbar_wait(&sm.bar_kv, 0, ac) && issue_s_dp(0);
-            for (int i = 0; ok && i < n_q; ++i) {
-                const int s = i % kStages;
-                const int b = i & 1;
-                if (i + 1 < n_q && !(ok = issue_s_dp(i + 1))) break;
-                const uint32_t q_addr = smem_u32(sm.q[s]);
-                const uint32_t do_addr = smem_u32(sm.dout[s]);
-                const uint32_t ds_addr = smem_u32(sm.ds[b]);
-                // dV += P^T dO
-                if (!(ok = mbar_wait(&sm.bar_p_full, i & 1, ac))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ts(tmem + C::kColDV, tmem + C::kColP + kk * 8, sw128_desc(do_addr + kk * 2048, 16384, 1024),
-                           kIdescKxMN, (i > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&sm.bar_dv_done);
-                // dK += dS^T Q
-                if (!(ok = mbar_wait(&sm.bar_ds_full[b], (i >> 1) & 1, ac))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
-                           sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN, (i > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(tmem + C::kColDP, sw128_desc(v_addr + kk * 32, 16, 1024),
+                               sw128_desc(do_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
+                    mma_commit(&sm.bar_dp_full);
                 }
-                // dQ = dS K, once the dQ warpgroup has copied out the previous one
-                if (i > 0 && !(ok = mbar_wait(&sm.bar_dq_free, (i - 1) & 1, ac))) break;
-                tc_fence_after();
+            } else if (warp == 2) {
+                // dV += P^T dO
+                for (int i = 0; ok && i < n_q; ++i) {
+                    const int s = i % kStages;
+                    if (!(ok = mbar_wait(&sm.bar_p_full, i & 1, ac))) break;
+                    tc_fence_after();
+                    const uint32_t do_addr = smem_u32(sm.dout[s]);
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
-                           sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
-                mma_commit(&sm.bar_dq_full);
-                mma_commit(&sm.bar_ds_empty[b]);
-                mma_commit(&sm.bar_qdo_empty[s]);
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_ts(tmem + C::kColDV, tmem + C::kColP + kk * 8, sw128_desc(do_addr + kk * 2048, 16384, 1024),
+                               kIdescKxMN, (i > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&sm.bar_dv_done);
+                    mma_commit(&sm.bar_qdo_empty[s]);
+                }
+                mma_commit(&sm.bar_dkdv_full);
+            } else if (warp == 3) {
+                // dK += dS^T Q
+                for (int i = 0; ok && i < n_q; ++i) {
+                    const int s = i % kStages;
+                    const int b = i & 1;
+                    if (!(ok = mbar_wait(&sm.bar_ds_full[b], (i >> 1) & 1, ac))) break;
+                    tc_fence_after();
+                    const uint32_t q_addr = smem_u32(sm.q[s]);
+                    const uint32_t ds_addr = smem_u32(sm.ds[b]);
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
+                               sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN, (i > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&sm.bar_ds_empty[b]);
+                    mma_commit(&sm.bar_qdo_empty[s]);
+                }
+                mma_commit(&sm.bar_dkdv_full);
             }
-            mma_commit(&sm.bar_dkdv_full);
-            mma_commit(&sm.bar_drain);
-            mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
+            if (warp >= 1) {
+                mma_commit(&sm.bar_drain);
+                mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
+            }
         }
     } else if (warp < 12) {
         regs_inc<184>();
@@ -247,21 +254,28 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_before();
             mbar_arrive(&sm.bar_sdp_free);             // S^T, dP^T columns may be overwritten now
 
+            // Blocked (key, query) pairs get score -inf, hence P = 0 and dS = 0 exactly.  Done as
+            // a separate pass so the arithmetic loop below stays one branch-free block.
             const bool need_mask = (qt == kt) || (W > 0 && qt * kTile + kTile - 1 >= k0 + W);
-            const uint32_t lse2_a = smem_u32(sm.lse2[s]) + h * 64 * 4;
-            const uint32_t dlt_a = smem_u32(sm.delta[s]) + h * 64 * 4;
+            if (need_mask) {
+                // Query columns that see this key form one range [c_lo, c_hi] (query >= key, and
+                // query < key + W under a window): an unsigned compare and a select per element.
+                const int c_lo = key - qc0;
+                const int c_hi = W > 0 ? key + W - 1 - qc0 : INT_MAX / 2;
+                const uint32_t span = (uint32_t)(c_hi - c_lo);
+#pragma unroll
+                for (int e = 0; e < 64; ++e)
+                    rs[e] = ((uint32_t)(e - c_lo) <= span) ? rs[e] : 0xff800000u;   // -inf
+            }
+            const float2* lse2 = reinterpret_cast<const float2*>(sm.lse2[s] + h * 64);
+            const float2* dlt = reinterpret_cast<const float2*>(sm.delta[s] + h * 64);
             uint32_t pk[32], dk[32];
 #pragma unroll
             for (int e = 0; e < 64; e += 2) {
-                const float2 ls = lds_f32x2(lse2_a + e * 4);
-                const float2 dl = lds_f32x2(dlt_a + e * 4);
-                float p0 = ex2_approx(fmaf(__uint_as_float(rs[e]), sl2, -ls.x));
-                float p1 = ex2_approx(fmaf(__uint_as_float(rs[e + 1]), sl2, -ls.y));
-                if (need_mask) {
-                    const int qa = qc0 + e;
-                    if (key > qa || (W > 0 && qa >= key + W)) p0 = 0.f;
-                    if (key > qa + 1 || (W > 0 && qa + 1 >= key + W)) p1 = 0.f;
-                }
+                const float2 ls = lse2[e >> 1];
+                const float2 dl = dlt[e >> 1];
+                const float p0 = ex2_approx(fmaf(__uint_as_float(rs[e]), sl2, -ls.x));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(rs[e + 1]), sl2, -ls.y));
                 const float d0 = p0 * (__uint_as_float(rd[e]) - dl.x);
                 const float d1 = p1 * (__uint_as_float(rd[e + 1]) - dl.y);
                 pk[e >> 1] = pack_bf16x2(p0, p1);
@@ -292,8 +306,27 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int r = wq * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
         bool ok = true;
+        bool issuer_ok = true;
+        const uint32_t k_addr = smem_u32(sm.k);
         for (int i = 0; i < n_q; ++i) {
             const int q = (qt_lo + i) * kTile + r;
+            if (warp == 12 && lane == 0 && issuer_ok) {
+                // dQ(i) = dS(i) K once dS(i) is in shared memory and this warpgroup has copied
+                // dQ(i-1) out of TMEM.
+                const int b = i & 1;
+                issuer_ok = mbar_wait(&sm.bar_ds_full[b], (i >> 1) & 1, ac) &&
+                            (i == 0 || mbar_wait(&sm.bar_dq_free, (i - 1) & 1, ac));
+                if (issuer_ok) {
+                    tc_fence_after();
+                    const uint32_t ds_addr = smem_u32(sm.ds[b]);
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
+                               sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
+                    mma_commit(&sm.bar_dq_full);
+                    mma_commit(&sm.bar_ds_empty[b]);
+                }
+            }
             if (!warp_wait(&sm.bar_dq_full, i & 1, ac)) { ok = false; break; }
             tc_fence_after();
             uint32_t rr[64];
@@ -309,6 +342,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     red_add_v4(dst + 4 * v4, __uint_as_float(rr[4 * v4]), __uint_as_float(rr[4 * v4 + 1]),
                                __uint_as_float(rr[4 * v4 + 2]), __uint_as_float(rr[4 * v4 + 3]));
             }
+        }
+        if (warp == 12 && lane == 0) {
+            mma_commit(&sm.bar_drain);
+            mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
         }
         // ---------------------------------------------------------- dK / dV epilogue (thread = key row)
         if (__all_sync(0xffffffffu, ok) && warp_wait(&sm.bar_dkdv_full, 0, ac)) {

@@ -9,7 +9,8 @@
 //   one CTA = one (batch*head, 256-query block) = two 128-row Q tiles sharing
 //   every K/V tile it loads; 12 warps:
 //     warp 0       TMA producer: Q0, Q1 once, then K_j / V_j through a ring
-//     warp 1       TMEM allocator and single-thread tcgen05.mma issuer
+//     warp 1       TMEM allocator; issues S0 = Q0 K_j^T and S1 = Q1 K_j^T
+//     warps 2, 3   issue O0 += P0 V_j and O1 += P1 V_j (one MMA stream per warp)
 //     warps 4..7   softmax warpgroup of Q tile 0 (thread r owns query row r)
 //     warps 8..11  softmax warpgroup of Q tile 1
 //   TMEM (512 columns):
@@ -17,9 +18,8 @@
 //     D = 128: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_t is written over S_t
 //   With separate P columns (D = 64) a softmax warpgroup hands its S columns back as
 //   soon as it has read them into registers, so the MMA warp computes S(j+1) while the
-//   exponentials of S(j) are still running; the issue order per key tile is
-//   S0(j+1) S1(j+1) PV0(j) PV1(j).  With P written over S (D = 128) the order is
-//   PV0(j) S0(j+1) PV1(j) S1(j+1) and each S waits for the PV that read its columns.
+//   exponentials of S(j) are still running.  With P written over S (D = 128)
+//   each S waits for the PV that read its columns.
 //
 // The running max is rescaled lazily: O and l are rescaled only when a row's max
 // grows by more than 8 (log2 units) over the max the exponentials use.  Every
@@ -30,6 +30,8 @@
 // of its first query, are never loaded for it; only the diagonal tile and the
 // window-edge tiles evaluate the visibility predicate.
 #pragma once
+
+#include <climits>
 
 #include "sm100.cuh"
 
@@ -112,8 +114,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     using C = FwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
-    FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(smem_align1024(smem_raw));
 
     constexpr int kStages = C::kStages;
     constexpr int kTileBytes = C::kTileBytes;
@@ -139,7 +140,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.bar_k[s], 1);
             mbar_init(&sm.bar_v[s], 1);
-            mbar_init(&sm.bar_kv_empty[s], 1);
+            mbar_init(&sm.bar_kv_empty[s], 3);        // S warp + two PV warps
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&sm.bar_s_full[t], 1);
@@ -147,7 +148,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&sm.bar_p_full[t], 128);
             mbar_init(&sm.bar_o_done[t], 1);
         }
-        mbar_init(&sm.bar_drain, 1);
+        mbar_init(&sm.bar_drain, 3);
         sm.abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -198,71 +199,71 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+    } else if (lane == 0) {
+        // ------------------------------------------------------------ MMA issuers
+        // One tcgen05.mma stream per warp: a single issuing thread cannot keep the
+        // tensor pipe busy with 128-row MMAs of N <= 128, several streams can.
+        //   warp 1: S0 = Q0 K_j^T and S1 = Q1 K_j^T
+        //   warp 2: O0 += P0 V_j        warp 3: O1 += P1 V_j
+        // Each of the three warps releases a K/V stage once its own MMAs on it are done.
+        auto active = [&](int j, int t) { return t ? (j >= lo1 && j <= hi1) : (j >= lo0 && j <= hi0); };
+        bool ok = true;
+        if (warp == 1) {
             const uint32_t q_addr0 = smem_u32(sm.q[0]), q_addr1 = smem_u32(sm.q[1]);
-            bool ok = mbar_wait(&sm.bar_q, 0, ac);
-            // S_t(j) = Q_t K_j^T into S_t's columns, once those columns are free.
-            auto issue_s = [&](int j, int t) -> bool {
-                const int i = j - (t ? lo1 : lo0);
+            ok = mbar_wait(&sm.bar_q, 0, ac);
+            for (int j = j_begin; ok && j <= j_end; ++j) {
                 const int it = j - j_begin;
                 const int s = it % kStages;
-                if (!mbar_wait(&sm.bar_k[s], (it / kStages) & 1, ac)) return false;
-                if (i > 0) {
-                    uint64_t* freed = C::kSeparateP ? &sm.bar_s_free[t] : &sm.bar_o_done[t];
-                    if (!mbar_wait(freed, (i - 1) & 1, ac)) return false;
-                }
-                tc_fence_after();
+                if (!(ok = mbar_wait(&sm.bar_k[s], (it / kStages) & 1, ac))) break;
                 const uint32_t k_addr = smem_u32(sm.k[s]);
-                const uint32_t q_addr = t ? q_addr1 : q_addr0;
-                const uint32_t col = t ? C::kColS1 : C::kColS0;
+                for (int t = 0; ok && t < 2; ++t) {
+                    if (!active(j, t)) continue;
+                    const int i = j - (t ? lo1 : lo0);
+                    if (i > 0) {
+                        // S_t shares TMEM with what the previous round still needs: the softmax copy of
+                        // S (separate P) or, when P is written over S, the PV MMA that reads it.
+                        uint64_t* freed = C::kSeparateP ? &sm.bar_s_free[t] : &sm.bar_o_done[t];
+                        if (!(ok = mbar_wait(freed, (i - 1) & 1, ac))) break;
+                    }
+                    tc_fence_after();
+                    const uint32_t q_addr = t ? q_addr1 : q_addr0;
+                    const uint32_t col = t ? C::kColS1 : C::kColS0;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_ss(tmem + col, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
-                           kIdescQK, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_ss(tmem + col, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
+                               kIdescQK, kk > 0);
+                    }
+                    mma_commit(&sm.bar_s_full[t]);
                 }
-                mma_commit(&sm.bar_s_full[t]);
-                return true;
-            };
-            // O_t += P_t V_j once the softmax warpgroup has written P_t(j).
-            auto issue_pv = [&](int j, int t) -> bool {
-                const int i = j - (t ? lo1 : lo0);
+                if (ok) mma_commit(&sm.bar_kv_empty[s]);
+            }
+        } else if (warp == 2 || warp == 3) {
+            const int t = warp - 2;
+            const uint32_t col_o = t ? C::kColO1 : C::kColO0;
+            const uint32_t col_p = t ? C::kColP1 : C::kColP0;
+            for (int j = j_begin; ok && j <= j_end; ++j) {
                 const int it = j - j_begin;
                 const int s = it % kStages;
-                if (!mbar_wait(&sm.bar_v[s], (it / kStages) & 1, ac)) return false;
-                if (!mbar_wait(&sm.bar_p_full[t], i & 1, ac)) return false;
+                if (!active(j, t)) {
+                    mbar_arrive(&sm.bar_kv_empty[s]);   // nothing of this warp reads stage s here
+                    continue;
+                }
+                const int i = j - (t ? lo1 : lo0);
+                if (!(ok = mbar_wait(&sm.bar_v[s], (it / kStages) & 1, ac))) break;
+                if (!(ok = mbar_wait(&sm.bar_p_full[t], i & 1, ac))) break;
                 tc_fence_after();
                 const uint32_t v_addr = smem_u32(sm.v[s]);
-                const uint32_t col_o = t ? C::kColO1 : C::kColO0;
-                const uint32_t col_p = t ? C::kColP1 : C::kColP0;
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk)
                     mma_ts(tmem + col_o, tmem + col_p + kk * 8, sw128_desc(v_addr + kk * 2048, 16384, 1024),
                            kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&sm.bar_o_done[t]);
-                return true;
-            };
-            auto active = [&](int j, int t) { return t ? (j >= lo1 && j <= hi1) : (j >= lo0 && j <= hi0); };
-
-            for (int t = 0; ok && t < 2; ++t)
-                if (active(j_begin, t)) ok = issue_s(j_begin, t);
-            for (int j = j_begin; ok && j <= j_end; ++j) {
-                if (C::kSeparateP) {
-                    for (int t = 0; ok && t < 2; ++t)
-                        if (j + 1 <= j_end && active(j + 1, t)) ok = issue_s(j + 1, t);
-                    for (int t = 0; ok && t < 2; ++t)
-                        if (active(j, t)) ok = issue_pv(j, t);
-                } else {
-                    for (int t = 0; ok && t < 2; ++t) {
-                        if (active(j, t)) ok = issue_pv(j, t);
-                        if (ok && j + 1 <= j_end && active(j + 1, t)) ok = issue_s(j + 1, t);
-                    }
-                }
-                if (ok) mma_commit(&sm.bar_kv_empty[(j - j_begin) % kStages]);
+                mma_commit(&sm.bar_kv_empty[s]);
             }
-            // Make sure no MMA is still running when TMEM is released.
+        }
+        if (warp <= 3) {
+            // No MMA of this warp may still be running when TMEM is released.
             mma_commit(&sm.bar_drain);
             mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
         }
@@ -306,16 +307,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             const bool need_mask = (j == qt) || (W > 0 && k0 <= qt * kTile + kTile - 1 - W);
             if (need_mask) {
+                // Visible columns of this row form one range [c_lo, c_hi]; one unsigned compare
+                // and a select per element, no per-element branch.
+                const int c_hi = i_abs - k0;
+                const int c_lo = W > 0 ? i_abs - W + 1 - k0 : INT_MIN / 2;
+                const uint32_t span = (uint32_t)(c_hi - c_lo);
 #pragma unroll
-                for (int e = 0; e < 128; ++e) {
-                    const int jj = k0 + e;
-                    if (jj > i_abs || (W > 0 && jj <= i_abs - W)) s[e] = -INFINITY;
-                }
+                for (int e = 0; e < 128; ++e)
+                    s[e] = ((uint32_t)(e - c_lo) <= span) ? s[e] : -INFINITY;
             }
-            float mx = fmax3(s[0], s[1], s[2]);
+            // Row max with four independent chains (short dependency chains).
+            float m0 = fmax3(s[0], s[1], s[2]), m1 = fmax3(s[3], s[4], s[5]);
+            float m2 = fmax3(s[6], s[7], s[8]), m3 = fmax3(s[9], s[10], s[11]);
 #pragma unroll
-            for (int e = 3; e < 127; e += 2) mx = fmax3(mx, s[e], s[e + 1]);
-            mx = fmaxf(mx, s[127]);
+            for (int e = 12; e < 120; e += 8) {
+                m0 = fmax3(m0, s[e], s[e + 1]);
+                m1 = fmax3(m1, s[e + 2], s[e + 3]);
+                m2 = fmax3(m2, s[e + 4], s[e + 5]);
+                m3 = fmax3(m3, s[e + 6], s[e + 7]);
+            }
+            m0 = fmax3(m0, s[124], s[125]);
+            m1 = fmax3(m1, s[126], s[127]);
+            m2 = fmax3(m2, s[120], s[121]);
+            m3 = fmax3(m3, s[122], s[123]);
+            const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
             const float m_new = mx * sl2;               // -inf stays -inf (sl2 > 0)
             const bool need = m_new > m_used + kLazyRescale;
             if (__any_sync(0xffffffffu, need)) {
