@@ -8,17 +8,18 @@
 //   16 warps:
 //     warp 0        TMA producer (Q, dO, lse, Delta rows through a 3-stage ring)
 //     warp 1        TMEM allocator; issues S^T = K Q^T and dP^T = V dO^T
-//     warp 2        issues dV += P^T dO        warp 3   issues dK += dS^T Q
+//     warp 2        issues dV += P^T dO        warp 3   issues dK += dS^T Q and dQ = dS K
 //     warps 4..7    P/dS warpgroup for query columns [0, 64) of each tile
 //     warps 8..11   P/dS warpgroup for query columns [64, 128)
-//     warps 12..15  dQ warpgroup: issues dQ = dS K, reads it out of TMEM and adds
-//                   it into the fp32 accumulator with vector reductions; at the
-//                   end writes dK (x scale) and dV
-//   Each MMA kind has its own issuing warp: one thread cannot issue 128-row
-//   MMAs of N <= 128 fast enough to keep the tensor pipe busy, four can.
+//     warps 12..15  dQ warpgroup: copies dQ(i) out of TMEM and adds it into the
+//                   fp32 accumulator (shared-memory staging + TMA bulk reduce-add);
+//                   at the end writes dK (x scale) and dV
+//   The MMAs are spread over three issuing warps: one thread cannot issue
+//   128-row MMAs of N <= 128 fast enough to keep the tensor pipe busy.
 //   TMEM (512 columns): S^T [0,128)  dP^T [128,256)  P^T bf16 [256,320)
 //                       dV [320,384)  dK [384,448)  dQ [448,512)
-//   Shared memory: K, V; 3 x (Q, dO, lse2, Delta); dS^T bf16 [key][query] x 2.
+//   Shared memory: K, V; 3 x (Q, dO, lse2, Delta); dS^T bf16 [key][query] x 2;
+//                  a 16 KB fp32 staging buffer for the dQ reduction.
 //
 // S(i+1) and dP(i+1) go in as soon as both P/dS warpgroups have copied S(i) and
 // dP(i) into registers, so the tensor pipe computes the next scores while the
@@ -45,6 +46,7 @@ struct Bwd64Smem {
     alignas(1024) uint8_t q[C::kStages][C::kTileBytes];
     alignas(1024) uint8_t dout[C::kStages][C::kTileBytes];
     alignas(1024) uint8_t ds[2][kTile * kTile * 2];          // dS^T bf16, two 64-query halves each
+    alignas(1024) uint8_t dq_stage[kTile * 32 * 4];          // fp32 [128 rows][32 cols], 128B-swizzled
     alignas(16) float lse2[C::kStages][kTile];
     alignas(16) float delta[C::kStages][kTile];
     uint64_t bar_kv;
@@ -60,6 +62,8 @@ struct Bwd64Smem {
     uint64_t bar_dq_full;
     uint64_t bar_dq_free;         // dQ(i) copied out of TMEM
     uint64_t bar_dkdv_full;
+    uint64_t bar_stage_full;      // the dQ warpgroup has written the staging buffer
+    uint64_t bar_stage_free;      // the bulk reduce has finished reading it
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -68,7 +72,7 @@ struct Bwd64Smem {
 __global__ void __launch_bounds__(kBwd64Threads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const BwdParams p) {
+                const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
     using C = Bwd64Cfg;
     constexpr int D = C::D;
     extern __shared__ uint8_t smem_raw[];
@@ -105,12 +109,14 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(&sm.bar_dv_done, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.bar_ds_full[b], 256);
-            mbar_init(&sm.bar_ds_empty[b], 2);      // dK warp + dQ issuer
+            mbar_init(&sm.bar_ds_empty[b], 1);      // after dQ(i) (dK(i) precedes it in the same stream)
         }
         mbar_init(&sm.bar_dq_full, 1);
         mbar_init(&sm.bar_dq_free, 128);
         mbar_init(&sm.bar_dkdv_full, 2);            // last dV + last dK
-        mbar_init(&sm.bar_drain, 4);                // the four MMA-issuing threads
+        mbar_init(&sm.bar_stage_full, 128);
+        mbar_init(&sm.bar_stage_free, 1);
+        mbar_init(&sm.bar_drain, 3);                // the three MMA-issuing threads
         sm.abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -161,7 +167,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // -------------------------------------------------------- MMA issuers
             // One tcgen05.mma stream per warp (a single issuing thread cannot keep the
             // tensor pipe busy with N <= 128 MMAs): warp 1 S^T and dP^T, warp 2 dV,
-            // warp 3 dK; dQ is issued by the dQ warpgroup itself.
+            // warp 3 dK and dQ.
             const uint32_t k_addr = smem_u32(sm.k);
             const uint32_t v_addr = smem_u32(sm.v);
             bool ok = true;
@@ -201,7 +207,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 mma_commit(&sm.bar_dkdv_full);
             } else if (warp == 3) {
-                // dK += dS^T Q
+                // dK += dS^T Q, then dQ = dS K once the dQ warpgroup has copied out dQ(i-1)
                 for (int i = 0; ok && i < n_q; ++i) {
                     const int s = i % kStages;
                     const int b = i & 1;
@@ -215,8 +221,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
                                sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN, (i > 0 || kk > 0) ? 1u : 0u);
                     }
-                    mma_commit(&sm.bar_ds_empty[b]);
                     mma_commit(&sm.bar_qdo_empty[s]);
+                    if (i > 0 && !(ok = mbar_wait(&sm.bar_dq_free, (i - 1) & 1, ac))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
+                               sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
+                    mma_commit(&sm.bar_dq_full);
+                    mma_commit(&sm.bar_ds_empty[b]);
                 }
                 mma_commit(&sm.bar_dkdv_full);
             }
@@ -306,27 +319,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int r = wq * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
         bool ok = true;
-        bool issuer_ok = true;
-        const uint32_t k_addr = smem_u32(sm.k);
         for (int i = 0; i < n_q; ++i) {
-            const int q = (qt_lo + i) * kTile + r;
-            if (warp == 12 && lane == 0 && issuer_ok) {
-                // dQ(i) = dS(i) K once dS(i) is in shared memory and this warpgroup has copied
-                // dQ(i-1) out of TMEM.
-                const int b = i & 1;
-                issuer_ok = mbar_wait(&sm.bar_ds_full[b], (i >> 1) & 1, ac) &&
-                            (i == 0 || mbar_wait(&sm.bar_dq_free, (i - 1) & 1, ac));
-                if (issuer_ok) {
-                    tc_fence_after();
-                    const uint32_t ds_addr = smem_u32(sm.ds[b]);
-#pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk)
-                        mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
-                               sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
-                    mma_commit(&sm.bar_dq_full);
-                    mma_commit(&sm.bar_ds_empty[b]);
-                }
-            }
             if (!warp_wait(&sm.bar_dq_full, i & 1, ac)) { ok = false; break; }
             tc_fence_after();
             uint32_t rr[64];
@@ -335,18 +328,29 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.bar_dq_free);
-            if (q < p.T) {
-                float* dst = p.dq_acc + ((size_t)bh * p.T + q) * D;
+            // Add dQ(i) into the fp32 accumulator: 32 columns at a time through the 16 KB staging
+            // buffer and a TMA bulk reduce-add of whole 128-byte rows (rows past T are skipped).
+            const uint32_t row_a = smem_u32(sm.dq_stage) + r * 128;
+            for (int hq = 0; hq < 2; ++hq) {
+                const int use = 2 * i + hq;             // uses of the staging buffer so far
+                if (use > 0 && !warp_wait(&sm.bar_stage_free, (use - 1) & 1, ac)) { ok = false; break; }
 #pragma unroll
-                for (int v4 = 0; v4 < 16; ++v4)
-                    red_add_v4(dst + 4 * v4, __uint_as_float(rr[4 * v4]), __uint_as_float(rr[4 * v4 + 1]),
-                               __uint_as_float(rr[4 * v4 + 2]), __uint_as_float(rr[4 * v4 + 3]));
+                for (int c = 0; c < 8; ++c)
+                    st_shared_v4(row_a + ((c ^ (r & 7)) << 4), rr[hq * 32 + 4 * c], rr[hq * 32 + 4 * c + 1],
+                                 rr[hq * 32 + 4 * c + 2], rr[hq * 32 + 4 * c + 3]);
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.bar_stage_full);
+                if (warp == 12 && lane == 0) {
+                    if (!mbar_wait(&sm.bar_stage_full, use & 1, ac)) { ok = false; break; }
+                    tma_reduce_add_3d(&tm_dq, sm.dq_stage, hq * 32, (qt_lo + i) * kTile, bh);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
+                    mbar_arrive(&sm.bar_stage_free);
+                }
             }
+            if (!ok) break;
         }
-        if (warp == 12 && lane == 0) {
-            mma_commit(&sm.bar_drain);
-            mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
-        }
+        if (warp == 12 && lane == 0) bulk_wait_group0();   // every reduce has landed in global memory
         // ---------------------------------------------------------- dK / dV epilogue (thread = key row)
         if (__all_sync(0xffffffffu, ok) && warp_wait(&sm.bar_dkdv_full, 0, ac)) {
             tc_fence_after();

@@ -316,21 +316,51 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int e = 0; e < 128; ++e)
                     s[e] = ((uint32_t)(e - c_lo) <= span) ? s[e] : -INFINITY;
             }
-            // Row max with four independent chains (short dependency chains).
-            float m0 = fmax3(s[0], s[1], s[2]), m1 = fmax3(s[3], s[4], s[5]);
-            float m2 = fmax3(s[6], s[7], s[8]), m3 = fmax3(s[9], s[10], s[11]);
+            // Exponentials.  After the first tile of a row the reference max m_used is finite and
+            // the exponentials start at once with it, the tile's own max being computed in the
+            // same pass.  Only if some row's max now exceeds m_used by more than the lazy-rescale
+            // margin (rare) is the tile redone below with the new max; nothing has been stored or
+            // accumulated at that point.
+            uint32_t pk[64];
+            float rs = 0.f;
+            float mx;
+            if (i == 0) {
+                // First tile of this warpgroup: its max becomes the reference (O is still empty).
+                float m0 = fmax3(s[0], s[1], s[2]), m1 = fmax3(s[3], s[4], s[5]);
+                float m2 = fmax3(s[6], s[7], s[8]), m3 = fmax3(s[9], s[10], s[11]);
 #pragma unroll
-            for (int e = 12; e < 120; e += 8) {
-                m0 = fmax3(m0, s[e], s[e + 1]);
-                m1 = fmax3(m1, s[e + 2], s[e + 3]);
-                m2 = fmax3(m2, s[e + 4], s[e + 5]);
-                m3 = fmax3(m3, s[e + 6], s[e + 7]);
+                for (int e = 12; e < 120; e += 8) {
+                    m0 = fmax3(m0, s[e], s[e + 1]);
+                    m1 = fmax3(m1, s[e + 2], s[e + 3]);
+                    m2 = fmax3(m2, s[e + 4], s[e + 5]);
+                    m3 = fmax3(m3, s[e + 6], s[e + 7]);
+                }
+                m0 = fmax3(m0, s[124], s[125]);
+                m1 = fmax3(m1, s[126], s[127]);
+                m2 = fmax3(m2, s[120], s[121]);
+                m3 = fmax3(m3, s[122], s[123]);
+                m_used = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;
             }
-            m0 = fmax3(m0, s[124], s[125]);
-            m1 = fmax3(m1, s[126], s[127]);
-            m2 = fmax3(m2, s[120], s[121]);
-            m3 = fmax3(m3, s[122], s[123]);
-            const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+            {
+                const float m_spec = (m_used == -INFINITY) ? 0.f : m_used;
+                float m0 = -INFINITY, m1 = -INFINITY;
+                float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+                for (int e = 0; e < 128; e += 4) {
+                    m0 = fmax3(m0, s[e], s[e + 1]);
+                    m1 = fmax3(m1, s[e + 2], s[e + 3]);
+                    const float a = ex2_approx(fmaf(s[e], sl2, -m_spec));
+                    const float b = ex2_approx(fmaf(s[e + 1], sl2, -m_spec));
+                    const float c = ex2_approx(fmaf(s[e + 2], sl2, -m_spec));
+                    const float d = ex2_approx(fmaf(s[e + 3], sl2, -m_spec));
+                    r0 += a + b;
+                    r1 += c + d;
+                    pk[e >> 1] = pack_bf16x2(a, b);
+                    pk[(e >> 1) + 1] = pack_bf16x2(c, d);
+                }
+                mx = fmaxf(m0, m1);
+                rs = r0 + r1;
+            }
             const float m_new = mx * sl2;               // -inf stays -inf (sl2 > 0)
             const bool need = m_new > m_used + kLazyRescale;
             if (__any_sync(0xffffffffu, need)) {
@@ -351,21 +381,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         tmem_st32(t_lane + col_o + c * 32, r);
                     }
                 }
-            }
-            const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
-            float rs0 = 0.f, rs1 = 0.f;
-            uint32_t pk[64];
+                // Redo this tile's exponentials against the new reference (rows that kept their
+                // reference recompute the same values).
+                const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
+                float r0 = 0.f, r1 = 0.f;
 #pragma unroll
-            for (int e = 0; e < 128; e += 2) {
-                float a = s[e], b = s[e + 1];
-                fma2_scale_sub(a, b, sl2, m_use);
-                a = ex2_approx(a);
-                b = ex2_approx(b);
-                rs0 += a;
-                rs1 += b;
-                pk[e >> 1] = pack_bf16x2(a, b);
+                for (int e = 0; e < 128; e += 2) {
+                    const float a = ex2_approx(fmaf(s[e], sl2, -m_use));
+                    const float b = ex2_approx(fmaf(s[e + 1], sl2, -m_use));
+                    r0 += a;
+                    r1 += b;
+                    pk[e >> 1] = pack_bf16x2(a, b);
+                }
+                rs = r0 + r1;
             }
-            l += rs0 + rs1;
+            l += rs;
             // Separate P columns: the previous PV must have finished reading them.
             if (C::kSeparateP && i > 0) {
                 if (!warp_wait(&sm.bar_o_done[t], (i - 1) & 1, ac)) { ok = false; break; }

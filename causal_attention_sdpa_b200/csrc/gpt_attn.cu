@@ -65,6 +65,21 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, int BH, int T, int D) {
     return r == CUDA_SUCCESS;
 }
 
+// fp32 dQ accumulator [BH, T, D] as a 3-D tensor (D, T, BH); 32-column x 128-row boxes
+// (128 bytes wide, 128-byte swizzle) for the bulk reduce-add.
+bool make_tmap_f32_acc(CUtensorMap* m, const void* base, int BH, int T, int D) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)T * D * 4};
+    cuuint32_t box[3] = {32, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
 int check_shape(int B, int H, int T, int D) {
@@ -164,9 +179,11 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
     p.timeout_ns = wait_timeout_ns();
     const unsigned grid = (unsigned)((long long)w.n_tiles * BH);
     if constexpr (D == 64) {
+        CUtensorMap mdq;
+        if (!make_tmap_f32_acc(&mdq, w.dq_acc, BH, T, D)) return GPT_ATTN_ERR_CUDA;
         const size_t smem = sizeof(Bwd64Smem) + 1024;
         if (!set_smem(attn_bwd_kernel, smem)) return GPT_ATTN_ERR_CUDA;
-        attn_bwd_kernel<<<grid, kBwd64Threads, smem, st>>>(mq, mk, mv, mdo, p);
+        attn_bwd_kernel<<<grid, kBwd64Threads, smem, st>>>(mq, mk, mv, mdo, mdq, p);
     } else {
         const size_t smem = sizeof(BwdSmem<D>) + 1024;
         if (!set_smem(attn_bwd_serial_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
