@@ -40,6 +40,7 @@ struct BwdParams {
     const float* lse2;      // [BH, T_pad]  lse * log2(e); +inf past T
     const float* delta;     // [BH, T_pad]  dO_i . O_i;    0 past T
     float* dq_acc;          // [BH, T, D]   fp32, zeroed by the prep kernel
+    int* sched;             // work-unit counter of the persistent kernel, zeroed by the prep kernel
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
     int T;
@@ -106,8 +107,10 @@ template <int D>
 __global__ void __launch_bounds__(256)
 attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                      const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ delta,
-                     float* __restrict__ dq_acc, int T, int T_pad, long long total_rows_pad) {
+                     float* __restrict__ dq_acc, int* __restrict__ sched, int T, int T_pad,
+                     long long total_rows_pad) {
     constexpr int G = D / 8;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0;
     const long long row = (long long)blockIdx.x * (256 / G) + threadIdx.x / G;
     const int g = threadIdx.x % G;
     const bool in_range = row < total_rows_pad;

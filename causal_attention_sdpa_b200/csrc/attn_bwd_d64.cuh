@@ -1,30 +1,37 @@
-// Pipelined backward kernel for head dimension 64 (the GPT-2 shapes).
+// Persistent pipelined backward kernel for head dimension 64 (the GPT-2 shapes).
 //
 // Same gradient and decomposition as attn_bwd.cuh (P, dV = P^T dO, dP, Delta,
-// dS = P (dP - Delta), dK, dQ), same work unit (one CTA per batch*head and
-// 128-key tile, K and V resident in shared memory, query tiles streamed), but
-// the five MMAs of query tile i overlap the P/dS arithmetic of tile i+1:
+// dS = P (dP - Delta), dK, dQ) and the same work unit: one (batch*head, 128-key
+// tile), whose K and V stay in shared memory while the query tiles that see it
+// stream past.  One CTA runs per SM and takes work units from a counter in the
+// workspace, in head-major order (the units of a head run close together, so its
+// Q, dO and dQ rows are served from L2).  K/V are double-buffered across units,
+// so the next unit's loads and first scores overlap the end of the current one.
 //
 //   16 warps:
-//     warp 0        TMA producer (Q, dO, lse, Delta rows through a 3-stage ring)
+//     warp 0        TMA producer: takes units, loads K/V and streams Q, dO, lse, Delta
 //     warp 1        TMEM allocator; issues S^T = K Q^T and dP^T = V dO^T
 //     warp 2        issues dV += P^T dO        warp 3   issues dK += dS^T Q and dQ = dS K
 //     warps 4..7    P/dS warpgroup for query columns [0, 64) of each tile
 //     warps 8..11   P/dS warpgroup for query columns [64, 128)
 //     warps 12..15  dQ warpgroup: copies dQ(i) out of TMEM and adds it into the
 //                   fp32 accumulator (shared-memory staging + TMA bulk reduce-add);
-//                   at the end writes dK (x scale) and dV
+//                   after each unit writes its dK (x scale) and dV
 //   The MMAs are spread over three issuing warps: one thread cannot issue
 //   128-row MMAs of N <= 128 fast enough to keep the tensor pipe busy.
 //   TMEM (512 columns): S^T [0,128)  dP^T [128,256)  P^T bf16 [256,320)
 //                       dV [320,384)  dK [384,448)  dQ [448,512)
-//   Shared memory: K, V; 3 x (Q, dO, lse2, Delta); dS^T bf16 [key][query] x 2;
+//   Shared memory: K, V x 2; 2 x (Q, dO, lse2, Delta); dS^T bf16 [key][query] x 2;
 //                  a 16 KB fp32 staging buffer for the dQ reduction.
 //
+// Every per-tile barrier phase counts query tiles over all units the CTA has
+// processed (g), so the pipeline runs on from one unit into the next.
 // S(i+1) and dP(i+1) go in as soon as both P/dS warpgroups have copied S(i) and
 // dP(i) into registers, so the tensor pipe computes the next scores while the
 // exponentials of this tile run.
 #pragma once
+
+#include <climits>
 
 #include "attn_bwd.cuh"
 
@@ -34,40 +41,61 @@ constexpr int kBwd64Threads = 512;
 
 struct Bwd64Cfg {
     static constexpr int D = 64;
-    static constexpr int kStages = 3;
+    static constexpr int kStages = 2;                        // Q/dO ring depth
     static constexpr int kTileBytes = kTile * D * 2;         // 16 KB
     static constexpr uint32_t kColS = 0, kColDP = 128, kColP = 256, kColDV = 320, kColDK = 384, kColDQ = 448;
+    // Threads that read each unit id: warps 1..3 (one lane each) + 256 P/dS + 128 dQ.
+    static constexpr uint32_t kUnitReaders = 3 + 256 + 128;
 };
 
 struct Bwd64Smem {
     using C = Bwd64Cfg;
-    alignas(1024) uint8_t k[C::kTileBytes];
-    alignas(1024) uint8_t v[C::kTileBytes];
+    alignas(1024) uint8_t k[2][C::kTileBytes];
+    alignas(1024) uint8_t v[2][C::kTileBytes];
     alignas(1024) uint8_t q[C::kStages][C::kTileBytes];
     alignas(1024) uint8_t dout[C::kStages][C::kTileBytes];
     alignas(1024) uint8_t ds[2][kTile * kTile * 2];          // dS^T bf16, two 64-query halves each
     alignas(1024) uint8_t dq_stage[kTile * 32 * 4];          // fp32 [128 rows][32 cols], 128B-swizzled
     alignas(16) float lse2[C::kStages][kTile];
     alignas(16) float delta[C::kStages][kTile];
-    uint64_t bar_kv;
+    int unit[2];                  // work-unit ring: id, or -1 when there is no more work
+    uint64_t bar_unit_full[2];
+    uint64_t bar_unit_empty[2];
+    uint64_t bar_kv_full[2];
+    uint64_t bar_kv_empty[2];     // S/dP warp and dK/dQ warp done with this K/V buffer
     uint64_t bar_qdo_full[C::kStages];
     uint64_t bar_qdo_empty[C::kStages];
     uint64_t bar_s_full;
     uint64_t bar_dp_full;
-    uint64_t bar_sdp_free;        // both P/dS warpgroups have S(i), dP(i) in registers
-    uint64_t bar_p_full;          // P^T(i) in TMEM
-    uint64_t bar_dv_done;         // dV(i) MMA finished: P^T columns free
-    uint64_t bar_ds_full[2];      // dS^T(i) in shared buffer i % 2
-    uint64_t bar_ds_empty[2];     // dK(i), dQ(i) finished with buffer i % 2
+    uint64_t bar_sdp_free;        // both P/dS warpgroups have S(g), dP(g) in registers
+    uint64_t bar_p_full;          // P^T(g) in TMEM
+    uint64_t bar_dv_done;         // dV(g) MMA finished: P^T columns free
+    uint64_t bar_ds_full[2];      // dS^T(g) in shared buffer g % 2
+    uint64_t bar_ds_empty[2];     // dK(g), dQ(g) finished with buffer g % 2
     uint64_t bar_dq_full;
-    uint64_t bar_dq_free;         // dQ(i) copied out of TMEM
-    uint64_t bar_dkdv_full;
+    uint64_t bar_dq_free;         // dQ(g) copied out of TMEM
+    uint64_t bar_dkdv_full;       // last dV and dK of a unit finished
+    uint64_t bar_dkdv_free;       // dK, dV of a unit copied out of TMEM
     uint64_t bar_stage_full;      // the dQ warpgroup has written the staging buffer
     uint64_t bar_stage_free;      // the bulk reduce has finished reading it
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort_flag;
 };
+
+struct Bwd64Unit {
+    int bh, kt, k0, qt_lo, n_q;
+};
+
+__device__ __forceinline__ Bwd64Unit bwd64_unit(int u, const BwdParams& p) {
+    Bwd64Unit w;
+    w.bh = u / p.n_tiles;
+    w.kt = u % p.n_tiles;
+    w.k0 = w.kt * kTile;
+    w.qt_lo = w.kt;
+    w.n_q = bwd_last_query_tile(w.kt, p.n_tiles, p.window) - w.qt_lo + 1;
+    return w;
+}
 
 __global__ void __launch_bounds__(kBwd64Threads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -87,17 +115,17 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // Blocks of one head are adjacent in launch order (its Q, dO and dQ rows stay in
-    // L2 across its key tiles); key tile 0 sees the most query tiles and launches first.
-    const int bh = blockIdx.x / p.n_tiles;
-    const int kt = blockIdx.x % p.n_tiles;
-    const int k0 = kt * kTile;
-    const int qt_lo = kt;
-    const int qt_hi = bwd_last_query_tile(kt, p.n_tiles, p.window);
-    const int n_q = qt_hi - qt_lo + 1;
+    const int total_units = p.BH * p.n_tiles;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sm.bar_kv, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.bar_unit_full[b], 1);
+            mbar_init(&sm.bar_unit_empty[b], C::kUnitReaders);
+            mbar_init(&sm.bar_kv_full[b], 1);
+            mbar_init(&sm.bar_kv_empty[b], 2);
+            mbar_init(&sm.bar_ds_full[b], 256);
+            mbar_init(&sm.bar_ds_empty[b], 1);      // after dQ(g) (dK(g) precedes it in the same stream)
+        }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.bar_qdo_full[s], 1);
             mbar_init(&sm.bar_qdo_empty[s], 2);     // dV warp + dK warp
@@ -107,13 +135,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(&sm.bar_sdp_free, 256);
         mbar_init(&sm.bar_p_full, 256);
         mbar_init(&sm.bar_dv_done, 1);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.bar_ds_full[b], 256);
-            mbar_init(&sm.bar_ds_empty[b], 1);      // after dQ(i) (dK(i) precedes it in the same stream)
-        }
         mbar_init(&sm.bar_dq_full, 1);
         mbar_init(&sm.bar_dq_free, 128);
-        mbar_init(&sm.bar_dkdv_full, 2);            // last dV + last dK
+        mbar_init(&sm.bar_dkdv_full, 2);            // last dV + last dK of the unit
+        mbar_init(&sm.bar_dkdv_free, 128);
         mbar_init(&sm.bar_stage_full, 128);
         mbar_init(&sm.bar_stage_free, 1);
         mbar_init(&sm.bar_drain, 3);                // the three MMA-issuing threads
@@ -131,8 +156,17 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tmem = sm.tmem_base;
     const AbortCtl ac{&sm.abort_flag, p.timeout_ns};
 
+    // Next work unit for a consumer role: waits for ring slot n % 2, reads it, releases it.
+    auto read_unit = [&](int n, int& u) -> bool {
+        const int slot = n & 1;
+        if (!mbar_wait(&sm.bar_unit_full[slot], (n >> 1) & 1, ac)) return false;
+        u = *reinterpret_cast<volatile int*>(&sm.unit[slot]);
+        mbar_arrive(&sm.bar_unit_empty[slot]);
+        return true;
+    };
+
     // Launched with 128 registers per thread (512 x 128 = 65536).  Warpgroup 0
-    // (producer, MMA, 2 idle warps) 56, the two P/dS warpgroups 184, the dQ
+    // (producer, MMA issuers) 56, the two P/dS warpgroups 184, the dQ
     // warpgroup 88: 128 x (56 + 184 + 184 + 88) = 65536.
     if (warp < 4) {
         regs_dec<56>();
@@ -142,101 +176,130 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_do);
-            mbar_arrive_expect_tx(&sm.bar_kv, 2 * kTileBytes);
-            tma_load_3d(sm.k, &tm_k, &sm.bar_kv, 0, k0, bh);
-            tma_load_3d(sm.v, &tm_v, &sm.bar_kv, 0, k0, bh);
-            int it = 0;
-            for (; it < n_q; ++it) {
-                const int s = it % kStages;
-                const int n = it / kStages;
-                if (n > 0 && !mbar_wait(&sm.bar_qdo_empty[s], (n - 1) & 1, ac)) break;
-                const int q0 = (qt_lo + it) * kTile;
-                mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + 2 * kTile * 4);
-                tma_load_3d(sm.q[s], &tm_q, &sm.bar_qdo_full[s], 0, q0, bh);
-                tma_load_3d(sm.dout[s], &tm_do, &sm.bar_qdo_full[s], 0, q0, bh);
-                const size_t roff = (size_t)bh * p.T_pad + q0;
-                bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
-                bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_qdo_full[s]);
+            int g = 0;                         // query tiles loaded so far
+            int n_kv = 0;                      // K/V buffers loaded so far
+            bool ok = true;
+            for (int n = 0; ok; ++n) {
+                const int slot = n & 1;
+                int u = atomicAdd(p.sched, 1);
+                if (u >= total_units) u = -1;
+                if (n >= 2 && !(ok = mbar_wait(&sm.bar_unit_empty[slot], ((n >> 1) - 1) & 1, ac))) break;
+                *reinterpret_cast<volatile int*>(&sm.unit[slot]) = u;
+                mbar_arrive(&sm.bar_unit_full[slot]);
+                if (u < 0) break;
+                const Bwd64Unit w = bwd64_unit(u, p);
+                const int kb = n & 1;
+                if (n >= 2 && !(ok = mbar_wait(&sm.bar_kv_empty[kb], ((n >> 1) - 1) & 1, ac))) break;
+                mbar_arrive_expect_tx(&sm.bar_kv_full[kb], 2 * kTileBytes);
+                tma_load_3d(sm.k[kb], &tm_k, &sm.bar_kv_full[kb], 0, w.k0, w.bh);
+                tma_load_3d(sm.v[kb], &tm_v, &sm.bar_kv_full[kb], 0, w.k0, w.bh);
+                n_kv = n + 1;
+                for (int i = 0; i < w.n_q; ++i, ++g) {
+                    const int s = g % kStages;
+                    const int m = g / kStages;
+                    if (m > 0 && !(ok = mbar_wait(&sm.bar_qdo_empty[s], (m - 1) & 1, ac))) break;
+                    const int q0 = (w.qt_lo + i) * kTile;
+                    mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + 2 * kTile * 4);
+                    tma_load_3d(sm.q[s], &tm_q, &sm.bar_qdo_full[s], 0, q0, w.bh);
+                    tma_load_3d(sm.dout[s], &tm_do, &sm.bar_qdo_full[s], 0, q0, w.bh);
+                    const size_t roff = (size_t)w.bh * p.T_pad + q0;
+                    bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
+                    bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_qdo_full[s]);
+                }
             }
             if (sm.abort_flag) {
-                mbar_wait_drain(&sm.bar_kv, 0, p.timeout_ns);
-                for (int r = (it > kStages ? it - kStages : 0); r < it; ++r)
+                // Let every load already issued land before the CTA exits.
+                for (int r = (n_kv > 2 ? n_kv - 2 : 0); r < n_kv; ++r)
+                    mbar_wait_drain(&sm.bar_kv_full[r & 1], (r >> 1) & 1, p.timeout_ns);
+                for (int r = (g > kStages ? g - kStages : 0); r < g; ++r)
                     mbar_wait_drain(&sm.bar_qdo_full[r % kStages], (r / kStages) & 1, p.timeout_ns);
             }
-        } else if (lane == 0) {
+        } else if (lane == 0 && warp >= 1) {
             // -------------------------------------------------------- MMA issuers
-            // One tcgen05.mma stream per warp (a single issuing thread cannot keep the
-            // tensor pipe busy with N <= 128 MMAs): warp 1 S^T and dP^T, warp 2 dV,
-            // warp 3 dK and dQ.
-            const uint32_t k_addr = smem_u32(sm.k);
-            const uint32_t v_addr = smem_u32(sm.v);
             bool ok = true;
-            if (warp == 1) {
-                ok = mbar_wait(&sm.bar_kv, 0, ac);
-                for (int i = 0; ok && i < n_q; ++i) {
-                    const int s = i % kStages;
-                    if (!(ok = mbar_wait(&sm.bar_qdo_full[s], (i / kStages) & 1, ac))) break;
-                    if (i > 0 && !(ok = mbar_wait(&sm.bar_sdp_free, (i - 1) & 1, ac))) break;
-                    tc_fence_after();
-                    const uint32_t q_addr = smem_u32(sm.q[s]);
-                    const uint32_t do_addr = smem_u32(sm.dout[s]);
+            int g = 0;
+            for (int n = 0; ok; ++n) {
+                int u;
+                if (!(ok = read_unit(n, u)) || u < 0) break;
+                const Bwd64Unit w = bwd64_unit(u, p);
+                const int kb = n & 1;
+                const uint32_t k_addr = smem_u32(sm.k[kb]);
+                const uint32_t v_addr = smem_u32(sm.v[kb]);
+                if (warp == 1) {
+                    if (!(ok = mbar_wait(&sm.bar_kv_full[kb], (n >> 1) & 1, ac))) break;
+                    for (int i = 0; i < w.n_q; ++i, ++g) {
+                        const int s = g % kStages;
+                        if (!(ok = mbar_wait(&sm.bar_qdo_full[s], (g / kStages) & 1, ac))) break;
+                        if (g > 0 && !(ok = mbar_wait(&sm.bar_sdp_free, (g - 1) & 1, ac))) break;
+                        tc_fence_after();
+                        const uint32_t q_addr = smem_u32(sm.q[s]);
+                        const uint32_t do_addr = smem_u32(sm.dout[s]);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tmem + C::kColS, sw128_desc(k_addr + kk * 32, 16, 1024),
-                               sw128_desc(q_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
-                    mma_commit(&sm.bar_s_full);
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            mma_ss(tmem + C::kColS, sw128_desc(k_addr + kk * 32, 16, 1024),
+                                   sw128_desc(q_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
+                        mma_commit(&sm.bar_s_full);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tmem + C::kColDP, sw128_desc(v_addr + kk * 32, 16, 1024),
-                               sw128_desc(do_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
-                    mma_commit(&sm.bar_dp_full);
-                }
-            } else if (warp == 2) {
-                // dV += P^T dO
-                for (int i = 0; ok && i < n_q; ++i) {
-                    const int s = i % kStages;
-                    if (!(ok = mbar_wait(&sm.bar_p_full, i & 1, ac))) break;
-                    tc_fence_after();
-                    const uint32_t do_addr = smem_u32(sm.dout[s]);
-#pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk)
-                        mma_ts(tmem + C::kColDV, tmem + C::kColP + kk * 8, sw128_desc(do_addr + kk * 2048, 16384, 1024),
-                               kIdescKxMN, (i > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(&sm.bar_dv_done);
-                    mma_commit(&sm.bar_qdo_empty[s]);
-                }
-                mma_commit(&sm.bar_dkdv_full);
-            } else if (warp == 3) {
-                // dK += dS^T Q, then dQ = dS K once the dQ warpgroup has copied out dQ(i-1)
-                for (int i = 0; ok && i < n_q; ++i) {
-                    const int s = i % kStages;
-                    const int b = i & 1;
-                    if (!(ok = mbar_wait(&sm.bar_ds_full[b], (i >> 1) & 1, ac))) break;
-                    tc_fence_after();
-                    const uint32_t q_addr = smem_u32(sm.q[s]);
-                    const uint32_t ds_addr = smem_u32(sm.ds[b]);
-#pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
-                               sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN, (i > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            mma_ss(tmem + C::kColDP, sw128_desc(v_addr + kk * 32, 16, 1024),
+                                   sw128_desc(do_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
+                        mma_commit(&sm.bar_dp_full);
                     }
-                    mma_commit(&sm.bar_qdo_empty[s]);
-                    if (i > 0 && !(ok = mbar_wait(&sm.bar_dq_free, (i - 1) & 1, ac))) break;
-                    tc_fence_after();
+                    if (ok) mma_commit(&sm.bar_kv_empty[kb]);
+                } else if (warp == 2) {
+                    // dV += P^T dO; the first one of a unit overwrites dV once the previous
+                    // unit's dV has been copied out.
+                    for (int i = 0; i < w.n_q; ++i, ++g) {
+                        const int s = g % kStages;
+                        if (!(ok = mbar_wait(&sm.bar_p_full, g & 1, ac))) break;
+                        if (i == 0 && n > 0 && !(ok = mbar_wait(&sm.bar_dkdv_free, (n - 1) & 1, ac))) break;
+                        tc_fence_after();
+                        const uint32_t do_addr = smem_u32(sm.dout[s]);
 #pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk)
-                        mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
-                               sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
-                    mma_commit(&sm.bar_dq_full);
-                    mma_commit(&sm.bar_ds_empty[b]);
+                        for (int kk = 0; kk < kTile / 16; ++kk)
+                            mma_ts(tmem + C::kColDV, tmem + C::kColP + kk * 8,
+                                   sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdescKxMN,
+                                   (i > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(&sm.bar_dv_done);
+                        mma_commit(&sm.bar_qdo_empty[s]);
+                    }
+                    if (ok) mma_commit(&sm.bar_dkdv_full);
+                } else if (warp == 3) {
+                    // dK += dS^T Q, then dQ = dS K once the dQ warpgroup has copied out dQ(g-1)
+                    for (int i = 0; i < w.n_q; ++i, ++g) {
+                        const int s = g % kStages;
+                        const int b = g & 1;
+                        if (!(ok = mbar_wait(&sm.bar_ds_full[b], (g >> 1) & 1, ac))) break;
+                        if (i == 0 && n > 0 && !(ok = mbar_wait(&sm.bar_dkdv_free, (n - 1) & 1, ac))) break;
+                        tc_fence_after();
+                        const uint32_t q_addr = smem_u32(sm.q[s]);
+                        const uint32_t ds_addr = smem_u32(sm.ds[b]);
+#pragma unroll
+                        for (int kk = 0; kk < kTile / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                            mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
+                                   sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN,
+                                   (i > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(&sm.bar_qdo_empty[s]);
+                        if (g > 0 && !(ok = mbar_wait(&sm.bar_dq_free, (g - 1) & 1, ac))) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < kTile / 16; ++kk)
+                            mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
+                                   sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
+                        mma_commit(&sm.bar_dq_full);
+                        mma_commit(&sm.bar_ds_empty[b]);
+                    }
+                    if (ok) {
+                        mma_commit(&sm.bar_dkdv_full);
+                        mma_commit(&sm.bar_kv_empty[kb]);
+                    }
                 }
-                mma_commit(&sm.bar_dkdv_full);
             }
-            if (warp >= 1) {
-                mma_commit(&sm.bar_drain);
-                mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
-            }
+            // No MMA of this thread may still be running when TMEM is released.
+            mma_commit(&sm.bar_drain);
+            mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
         }
     } else if (warp < 12) {
         regs_inc<184>();
@@ -244,74 +307,80 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int h = (warp - 4) >> 2;              // query-column half of this warpgroup
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
-        const int key = k0 + r;
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
         const int W = p.window;
         const float sl2 = p.scale_log2;
         bool ok = true;
-        for (int i = 0; i < n_q; ++i) {
-            const int s = i % kStages;
-            const int b = i & 1;
-            const int qt = qt_lo + i;
-            const int qc0 = qt * kTile + h * 64;       // first query column of this half
-            if (!warp_wait(&sm.bar_qdo_full[s], (i / kStages) & 1, ac)) { ok = false; break; }
-            if (!warp_wait(&sm.bar_s_full, i & 1, ac)) { ok = false; break; }
-            if (!warp_wait(&sm.bar_dp_full, i & 1, ac)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t rs[64], rd[64];
-            tmem_ld32(t_lane + C::kColS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
-            tmem_ld32(t_lane + C::kColS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
-            tmem_ld32(t_lane + C::kColDP + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&rd[0]));
-            tmem_ld32(t_lane + C::kColDP + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rd[32]));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&sm.bar_sdp_free);             // S^T, dP^T columns may be overwritten now
+        int g = 0;
+        for (int n = 0; ok; ++n) {
+            int u = -1;
+            ok = __all_sync(0xffffffffu, read_unit(n, u));
+            if (!ok || u < 0) break;
+            const Bwd64Unit w = bwd64_unit(u, p);
+            const int key = w.k0 + r;
+            for (int i = 0; i < w.n_q; ++i, ++g) {
+                const int s = g % kStages;
+                const int b = g & 1;
+                const int qt = w.qt_lo + i;
+                const int qc0 = qt * kTile + h * 64;       // first query column of this half
+                if (!warp_wait(&sm.bar_qdo_full[s], (g / kStages) & 1, ac)) { ok = false; break; }
+                if (!warp_wait(&sm.bar_s_full, g & 1, ac)) { ok = false; break; }
+                if (!warp_wait(&sm.bar_dp_full, g & 1, ac)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t rs[64], rd[64];
+                tmem_ld32(t_lane + C::kColS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
+                tmem_ld32(t_lane + C::kColS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
+                tmem_ld32(t_lane + C::kColDP + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&rd[0]));
+                tmem_ld32(t_lane + C::kColDP + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rd[32]));
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&sm.bar_sdp_free);             // S^T, dP^T columns may be overwritten now
 
-            // Blocked (key, query) pairs get score -inf, hence P = 0 and dS = 0 exactly.  Done as
-            // a separate pass so the arithmetic loop below stays one branch-free block.
-            const bool need_mask = (qt == kt) || (W > 0 && qt * kTile + kTile - 1 >= k0 + W);
-            if (need_mask) {
-                // Query columns that see this key form one range [c_lo, c_hi] (query >= key, and
-                // query < key + W under a window): an unsigned compare and a select per element.
-                const int c_lo = key - qc0;
-                const int c_hi = W > 0 ? key + W - 1 - qc0 : INT_MAX / 2;
-                const uint32_t span = (uint32_t)(c_hi - c_lo);
+                // Blocked (key, query) pairs get score -inf, hence P = 0 and dS = 0 exactly.  Done as
+                // a separate pass so the arithmetic loop below stays one branch-free block.
+                const bool need_mask = (qt == w.kt) || (W > 0 && qt * kTile + kTile - 1 >= w.k0 + W);
+                if (need_mask) {
+                    // Query columns that see this key form one range [c_lo, c_hi] (query >= key, and
+                    // query < key + W under a window): an unsigned compare and a select per element.
+                    const int c_lo = key - qc0;
+                    const int c_hi = W > 0 ? key + W - 1 - qc0 : INT_MAX / 2;
+                    const uint32_t span = (uint32_t)(c_hi - c_lo);
 #pragma unroll
-                for (int e = 0; e < 64; ++e)
-                    rs[e] = ((uint32_t)(e - c_lo) <= span) ? rs[e] : 0xff800000u;   // -inf
+                    for (int e = 0; e < 64; ++e)
+                        rs[e] = ((uint32_t)(e - c_lo) <= span) ? rs[e] : 0xff800000u;   // -inf
+                }
+                const float2* lse2 = reinterpret_cast<const float2*>(sm.lse2[s] + h * 64);
+                const float2* dlt = reinterpret_cast<const float2*>(sm.delta[s] + h * 64);
+                uint32_t pk[32], dk[32];
+#pragma unroll
+                for (int e = 0; e < 64; e += 2) {
+                    const float2 ls = lse2[e >> 1];
+                    const float2 dl = dlt[e >> 1];
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(rs[e]), sl2, -ls.x));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(rs[e + 1]), sl2, -ls.y));
+                    const float d0 = p0 * (__uint_as_float(rd[e]) - dl.x);
+                    const float d1 = p1 * (__uint_as_float(rd[e + 1]) - dl.y);
+                    pk[e >> 1] = pack_bf16x2(p0, p1);
+                    dk[e >> 1] = pack_bf16x2(d0, d1);
+                }
+                // P^T(g) into TMEM once dV(g-1) has finished reading P^T(g-1)
+                if (g > 0 && !warp_wait(&sm.bar_dv_done, (g - 1) & 1, ac)) { ok = false; break; }
+                tc_fence_after();
+                tmem_st32(t_lane + C::kColP + h * 32, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sm.bar_p_full);
+                // dS^T(g) into shared buffer b once dK(g-2), dQ(g-2) have finished with it.
+                // Row r of half h holds queries [64h, 64h + 64): 8 chunks of 16 bytes, swizzled by row.
+                if (g >= 2 && !warp_wait(&sm.bar_ds_empty[b], ((g >> 1) - 1) & 1, ac)) { ok = false; break; }
+                const uint32_t row_a = smem_u32(sm.ds[b]) + h * 16384 + r * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    st_shared_v4(row_a + ((c ^ (r & 7)) << 4), dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.bar_ds_full[b]);
             }
-            const float2* lse2 = reinterpret_cast<const float2*>(sm.lse2[s] + h * 64);
-            const float2* dlt = reinterpret_cast<const float2*>(sm.delta[s] + h * 64);
-            uint32_t pk[32], dk[32];
-#pragma unroll
-            for (int e = 0; e < 64; e += 2) {
-                const float2 ls = lse2[e >> 1];
-                const float2 dl = dlt[e >> 1];
-                const float p0 = ex2_approx(fmaf(__uint_as_float(rs[e]), sl2, -ls.x));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(rs[e + 1]), sl2, -ls.y));
-                const float d0 = p0 * (__uint_as_float(rd[e]) - dl.x);
-                const float d1 = p1 * (__uint_as_float(rd[e + 1]) - dl.y);
-                pk[e >> 1] = pack_bf16x2(p0, p1);
-                dk[e >> 1] = pack_bf16x2(d0, d1);
-            }
-            // P^T(i) into TMEM once dV(i-1) has finished reading P^T(i-1)
-            if (i > 0 && !warp_wait(&sm.bar_dv_done, (i - 1) & 1, ac)) { ok = false; break; }
-            tc_fence_after();
-            tmem_st32(t_lane + C::kColP + h * 32, pk);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&sm.bar_p_full);
-            // dS^T(i) into shared buffer b once dK(i-2), dQ(i-2) have finished with it.
-            // Row r of half h holds queries [64h, 64h + 64): 8 chunks of 16 bytes, swizzled by row.
-            if (i >= 2 && !warp_wait(&sm.bar_ds_empty[b], ((i >> 1) - 1) & 1, ac)) { ok = false; break; }
-            const uint32_t row_a = smem_u32(sm.ds[b]) + h * 16384 + r * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_shared_v4(row_a + ((c ^ (r & 7)) << 4), dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.bar_ds_full[b]);
         }
-        (void)ok;
     } else {
         regs_dec<88>();
         // ------------------------------------------------------------ dQ warpgroup (thread = query / key row)
@@ -319,44 +388,51 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int r = wq * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
         bool ok = true;
-        for (int i = 0; i < n_q; ++i) {
-            if (!warp_wait(&sm.bar_dq_full, i & 1, ac)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t rr[64];
-            tmem_ld32(t_lane + C::kColDQ, *reinterpret_cast<uint32_t(*)[32]>(&rr[0]));
-            tmem_ld32(t_lane + C::kColDQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&rr[32]));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&sm.bar_dq_free);
-            // Add dQ(i) into the fp32 accumulator: 32 columns at a time through the 16 KB staging
-            // buffer and a TMA bulk reduce-add of whole 128-byte rows (rows past T are skipped).
-            const uint32_t row_a = smem_u32(sm.dq_stage) + r * 128;
-            for (int hq = 0; hq < 2; ++hq) {
-                const int use = 2 * i + hq;             // uses of the staging buffer so far
-                if (use > 0 && !warp_wait(&sm.bar_stage_free, (use - 1) & 1, ac)) { ok = false; break; }
+        int g = 0;
+        for (int n = 0; ok; ++n) {
+            int u = -1;
+            ok = __all_sync(0xffffffffu, read_unit(n, u));
+            if (!ok || u < 0) break;
+            const Bwd64Unit w = bwd64_unit(u, p);
+            for (int i = 0; i < w.n_q; ++i, ++g) {
+                if (!warp_wait(&sm.bar_dq_full, g & 1, ac)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t rr[64];
+                tmem_ld32(t_lane + C::kColDQ, *reinterpret_cast<uint32_t(*)[32]>(&rr[0]));
+                tmem_ld32(t_lane + C::kColDQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&rr[32]));
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&sm.bar_dq_free);
+                // Add dQ(g) into the fp32 accumulator: 32 columns at a time through the 16 KB staging
+                // buffer and a TMA bulk reduce-add of whole 128-byte rows (rows past T are skipped).
+                const uint32_t row_a = smem_u32(sm.dq_stage) + r * 128;
+                for (int hq = 0; hq < 2; ++hq) {
+                    const int use = 2 * g + hq;             // uses of the staging buffer so far
+                    if (use > 0 && !warp_wait(&sm.bar_stage_free, (use - 1) & 1, ac)) { ok = false; break; }
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    st_shared_v4(row_a + ((c ^ (r & 7)) << 4), rr[hq * 32 + 4 * c], rr[hq * 32 + 4 * c + 1],
-                                 rr[hq * 32 + 4 * c + 2], rr[hq * 32 + 4 * c + 3]);
-                fence_proxy_async_smem();
-                mbar_arrive(&sm.bar_stage_full);
-                if (warp == 12 && lane == 0) {
-                    if (!mbar_wait(&sm.bar_stage_full, use & 1, ac)) { ok = false; break; }
-                    tma_reduce_add_3d(&tm_dq, sm.dq_stage, hq * 32, (qt_lo + i) * kTile, bh);
-                    bulk_commit_group();
-                    bulk_wait_group_read0();
-                    mbar_arrive(&sm.bar_stage_free);
+                    for (int c = 0; c < 8; ++c)
+                        st_shared_v4(row_a + ((c ^ (r & 7)) << 4), rr[hq * 32 + 4 * c], rr[hq * 32 + 4 * c + 1],
+                                     rr[hq * 32 + 4 * c + 2], rr[hq * 32 + 4 * c + 3]);
+                    fence_proxy_async_smem();
+                    mbar_arrive(&sm.bar_stage_full);
+                    if (warp == 12 && lane == 0) {
+                        if (!mbar_wait(&sm.bar_stage_full, use & 1, ac)) { ok = false; break; }
+                        tma_reduce_add_3d(&tm_dq, sm.dq_stage, hq * 32, (w.qt_lo + i) * kTile, w.bh);
+                        bulk_commit_group();
+                        bulk_wait_group_read0();
+                        mbar_arrive(&sm.bar_stage_free);
+                    }
                 }
+                if (!ok) break;
             }
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
-        }
-        if (warp == 12 && lane == 0) bulk_wait_group0();   // every reduce has landed in global memory
-        // ---------------------------------------------------------- dK / dV epilogue (thread = key row)
-        if (__all_sync(0xffffffffu, ok) && warp_wait(&sm.bar_dkdv_full, 0, ac)) {
+            // ---------------------------------------------------------- dK / dV of this unit (thread = key row)
+            if (!warp_wait(&sm.bar_dkdv_full, n & 1, ac)) { ok = false; break; }
             tc_fence_after();
-            const int key = k0 + r;
+            const int key = w.k0 + r;
             const bool store = key < p.T;
-            const size_t off = ((size_t)bh * p.T + (store ? key : 0)) * D;
+            const size_t off = ((size_t)w.bh * p.T + (store ? key : 0)) * D;
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
                 __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + off;
@@ -379,7 +455,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&sm.bar_dkdv_free);
         }
+        if (warp == 12 && lane == 0) bulk_wait_group0();   // every reduce has landed in global memory
     }
 
     tc_fence_before();

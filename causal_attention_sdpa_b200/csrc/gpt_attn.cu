@@ -126,10 +126,13 @@ struct WsLayout {
     float* dq_acc;
     float* lse2;
     float* delta;
+    int* sched;
     int n_tiles;
     int T_pad;
 };
 
+// Workspace: fp32 dQ accumulator [BH, T, D] | lse*log2(e) [BH, T_pad] | Delta [BH, T_pad] |
+// 16 bytes holding the persistent kernel's work-unit counter.
 WsLayout ws_layout(void* ws, int BH, int T, int D) {
     WsLayout w;
     w.n_tiles = (T + kTile - 1) / kTile;
@@ -137,7 +140,20 @@ WsLayout ws_layout(void* ws, int BH, int T, int D) {
     w.dq_acc = static_cast<float*>(ws);
     w.lse2 = w.dq_acc + (size_t)BH * T * D;
     w.delta = w.lse2 + (size_t)BH * w.T_pad;
+    w.sched = reinterpret_cast<int*>(w.delta + (size_t)BH * w.T_pad);
     return w;
+}
+
+int sm_count() {
+    static int counts[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (counts[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        counts[dev] = n;
+    }
+    return counts[dev];
 }
 
 int launch_bwd_delta(const void* o, const float* lse, const void* dout, int BH, int T, int D, void* ws,
@@ -149,9 +165,11 @@ int launch_bwd_delta(const void* o, const float* lse, const void* dout, int BH, 
     const auto* o16 = static_cast<const __nv_bfloat16*>(o);
     const auto* do16 = static_cast<const __nv_bfloat16*>(dout);
     if (D == 64)
-        attn_bwd_prep_kernel<64><<<grid, 256, 0, st>>>(o16, do16, lse, w.lse2, w.delta, w.dq_acc, T, w.T_pad, rows);
+        attn_bwd_prep_kernel<64><<<grid, 256, 0, st>>>(o16, do16, lse, w.lse2, w.delta, w.dq_acc, w.sched, T,
+                                                        w.T_pad, rows);
     else
-        attn_bwd_prep_kernel<128><<<grid, 256, 0, st>>>(o16, do16, lse, w.lse2, w.delta, w.dq_acc, T, w.T_pad, rows);
+        attn_bwd_prep_kernel<128><<<grid, 256, 0, st>>>(o16, do16, lse, w.lse2, w.delta, w.dq_acc, w.sched, T,
+                                                         w.T_pad, rows);
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
@@ -167,6 +185,7 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
     p.lse2 = w.lse2;
     p.delta = w.delta;
     p.dq_acc = w.dq_acc;
+    p.sched = w.sched;
     p.dk = static_cast<__nv_bfloat16*>(dk);
     p.dv = static_cast<__nv_bfloat16*>(dv);
     p.T = T;
@@ -177,13 +196,16 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
     p.scale_log2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.timeout_ns = wait_timeout_ns();
-    const unsigned grid = (unsigned)((long long)w.n_tiles * BH);
+    const long long units = (long long)w.n_tiles * BH;
+    const unsigned grid = (unsigned)units;
     if constexpr (D == 64) {
         CUtensorMap mdq;
         if (!make_tmap_f32_acc(&mdq, w.dq_acc, BH, T, D)) return GPT_ATTN_ERR_CUDA;
         const size_t smem = sizeof(Bwd64Smem) + 1024;
         if (!set_smem(attn_bwd_kernel, smem)) return GPT_ATTN_ERR_CUDA;
-        attn_bwd_kernel<<<grid, kBwd64Threads, smem, st>>>(mq, mk, mv, mdo, mdq, p);
+        // persistent: one CTA per SM, work units taken from the counter in the workspace
+        const unsigned pgrid = (unsigned)(units < sm_count() ? units : sm_count());
+        attn_bwd_kernel<<<pgrid, kBwd64Threads, smem, st>>>(mq, mk, mv, mdo, mdq, p);
     } else {
         const size_t smem = sizeof(BwdSmem<D>) + 1024;
         if (!set_smem(attn_bwd_serial_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
@@ -273,7 +295,7 @@ size_t gpt_attn_bwd_workspace_bytes(int B, int H, int T, int D) {
     if (check_shape(B, H, T, D) != GPT_ATTN_OK) return 0;
     const size_t bh = (size_t)B * H;
     const size_t t_pad = ((size_t)T + 127) / 128 * 128;
-    return 4 * (bh * T * D + 2 * bh * t_pad);
+    return 4 * (bh * T * D + 2 * bh * t_pad) + 16;
 }
 
 int gpt_attn_bwd_delta(const void* o, const float* lse, const void* dO, int B, int H, int T, int D,

@@ -66,8 +66,10 @@ int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
 /*
  * Bytes of device workspace gpt_attn_bwd needs for this shape: an fp32 dQ
- * accumulator [B, H, T, D] plus two fp32 row vectors per head padded to a
- * multiple of 128 rows (the log2-scaled lse and Delta_i = dO_i . O_i).
+ * accumulator [B, H, T, D], two fp32 row vectors per head padded to a
+ * multiple of 128 rows (the log2-scaled lse and Delta_i = dO_i . O_i), and
+ * 16 bytes for the work-unit counter of the backward kernel:
+ * 4 * (B*H*T*D + 2*B*H*T_pad) + 16 with T_pad = ceil(T / 128) * 128.
  * Returns 0 for shapes gpt_attn_bwd would reject.
  */
 size_t gpt_attn_bwd_workspace_bytes(int B, int H, int T, int D);

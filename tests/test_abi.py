@@ -76,9 +76,9 @@ def test_fwd_misaligned(L, which):
 
 
 def test_workspace_bytes(L):
-    # fp32 dQ accumulator + two fp32 rows per head padded to a multiple of 128
-    assert ga.gpt_attn_bwd_workspace_bytes(2, 3, 200, 64) == 4 * (6 * 200 * 64 + 2 * 6 * 256)
-    assert ga.gpt_attn_bwd_workspace_bytes(1, 1, 128, 128) == 4 * (128 * 128 + 2 * 128)
+    # fp32 dQ accumulator + two fp32 rows per head padded to a multiple of 128 + a 16-byte counter
+    assert ga.gpt_attn_bwd_workspace_bytes(2, 3, 200, 64) == 4 * (6 * 200 * 64 + 2 * 6 * 256) + 16
+    assert ga.gpt_attn_bwd_workspace_bytes(1, 1, 128, 128) == 4 * (128 * 128 + 2 * 128) + 16
     assert ga.gpt_attn_bwd_workspace_bytes(1, 1, 8, 32) == 0
     assert ga.gpt_attn_bwd_workspace_bytes(0, 1, 8, 64) == 0
 
