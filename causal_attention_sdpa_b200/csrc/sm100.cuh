@@ -281,23 +281,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// 2^x on the FMA pipe, to take part of the exponentials off the MUFU unit.
-// x = j + f with j = round(x) (the 1.5 * 2^23 addition leaves it in the low mantissa
-// bits) and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted by relative-error
-// minimax (Remez exchange, csrc/gen_exp2_poly.py; max relative error 7.5e-5, far below
-// the bf16 rounding of P); j is added to the exponent field.  x < -125 returns 0
-// (this covers masked scores at -inf).  Valid for x <= 127.
-__device__ __forceinline__ float ex2_poly(float x) {
-    const float xc = fmaxf(x, -125.0f);
-    const float t = xc + 12582912.0f;
-    const float f = xc - (t - 12582912.0f);
-    float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
-    p = fmaf(p, f, 0.6932609677314758f);
-    p = fmaf(p, f, 0.9999280571937561f);
-    const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-    return x < -125.0f ? 0.0f : r;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
