@@ -14,15 +14,15 @@
 //     warp 2        issues dV += P^T dO        warp 3   issues dK += dS^T Q and dQ = dS K
 //     warps 4..7    P/dS warpgroup for query columns [0, 64) of each tile
 //     warps 8..11   P/dS warpgroup for query columns [64, 128)
-//     warps 12..15  dQ warpgroup: copies dQ(i) out of TMEM and adds it into the
-//                   fp32 accumulator (shared-memory staging + TMA bulk reduce-add);
-//                   after each unit writes its dK (x scale) and dV
+//     warps 12..15  dQ warpgroup: copies dQ(g) out of TMEM and adds it into the
+//                   fp32 accumulator (staged in the dS buffer dQ(g) has just read,
+//                   then TMA bulk reduce-add); writes each unit's dK (x scale) and dV
 //   The MMAs are spread over three issuing warps: one thread cannot issue
 //   128-row MMAs of N <= 128 fast enough to keep the tensor pipe busy.
 //   TMEM (512 columns): S^T [0,128)  dP^T [128,256)  P^T bf16 [256,320)
 //                       dV [320,384)  dK [384,448)  dQ [448,512)
-//   Shared memory: K, V x 2; 2 x (Q, dO, lse2, Delta); dS^T bf16 [key][query] x 2;
-//                  a 16 KB fp32 staging buffer for the dQ reduction.
+//   Shared memory: K, V x 2; 2 x (Q, dO, lse2, Delta); dS^T bf16 [key][query] x 2
+//                  (each doubles as the fp32 staging of dQ for its reduction).
 //
 // Every per-tile barrier phase counts query tiles over all units the CTA has
 // processed (g), so the pipeline runs on from one unit into the next.
@@ -54,8 +54,9 @@ struct Bwd64Smem {
     alignas(1024) uint8_t v[2][C::kTileBytes];
     alignas(1024) uint8_t q[C::kStages][C::kTileBytes];
     alignas(1024) uint8_t dout[C::kStages][C::kTileBytes];
-    alignas(1024) uint8_t ds[2][kTile * kTile * 2];          // dS^T bf16, two 64-query halves each
-    alignas(1024) uint8_t dq_stage[kTile * 32 * 4];          // fp32 [128 rows][32 cols], 128B-swizzled
+    // dS^T bf16 [key][query] as two 64-query halves; once dK(g) and dQ(g) have read it, the same
+    // 32 KB stages dQ(g) in fp32 as two [128 rows][32 cols] 128B-swizzled boxes for the reduce.
+    alignas(1024) uint8_t ds[2][kTile * kTile * 2];
     alignas(16) float lse2[C::kStages][kTile];
     alignas(16) float delta[C::kStages][kTile];
     int unit[2];                  // work-unit ring: id, or -1 when there is no more work
@@ -71,13 +72,12 @@ struct Bwd64Smem {
     uint64_t bar_p_full;          // P^T(g) in TMEM
     uint64_t bar_dv_done;         // dV(g) MMA finished: P^T columns free
     uint64_t bar_ds_full[2];      // dS^T(g) in shared buffer g % 2
-    uint64_t bar_ds_empty[2];     // dK(g), dQ(g) finished with buffer g % 2
+    uint64_t bar_ds_empty[2];     // buffer g % 2 free again: dK(g), dQ(g) read it, dQ(g) staged and reduced
     uint64_t bar_dq_full;
     uint64_t bar_dq_free;         // dQ(g) copied out of TMEM
     uint64_t bar_dkdv_full;       // last dV and dK of a unit finished
     uint64_t bar_dkdv_free;       // dK, dV of a unit copied out of TMEM
-    uint64_t bar_stage_full;      // the dQ warpgroup has written the staging buffer
-    uint64_t bar_stage_free;      // the bulk reduce has finished reading it
+    uint64_t bar_stage_full;      // the dQ warpgroup has staged dQ(g)
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -124,7 +124,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&sm.bar_kv_full[b], 1);
             mbar_init(&sm.bar_kv_empty[b], 2);
             mbar_init(&sm.bar_ds_full[b], 256);
-            mbar_init(&sm.bar_ds_empty[b], 1);      // after dQ(g) (dK(g) precedes it in the same stream)
+            mbar_init(&sm.bar_ds_empty[b], 1);      // by the dQ reduce issuer
         }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.bar_qdo_full[s], 1);
@@ -140,7 +140,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(&sm.bar_dkdv_full, 2);            // last dV + last dK of the unit
         mbar_init(&sm.bar_dkdv_free, 128);
         mbar_init(&sm.bar_stage_full, 128);
-        mbar_init(&sm.bar_stage_free, 1);
         mbar_init(&sm.bar_drain, 3);                // the three MMA-issuing threads
         sm.abort_flag = 0;
         fence_barrier_init();
@@ -288,8 +287,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         for (int kk = 0; kk < kTile / 16; ++kk)
                             mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
                                    sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
-                        mma_commit(&sm.bar_dq_full);
-                        mma_commit(&sm.bar_ds_empty[b]);
+                        mma_commit(&sm.bar_dq_full);      // dK(g) precedes dQ(g): both done when this fires
                     }
                     if (ok) {
                         mma_commit(&sm.bar_dkdv_full);
@@ -394,69 +392,76 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ok = __all_sync(0xffffffffu, read_unit(n, u));
             if (!ok || u < 0) break;
             const Bwd64Unit w = bwd64_unit(u, p);
+            // dK / dV of this unit (thread = key row): copied out as soon as the unit's last dQ is
+            // complete, before that dQ is reduced, so the next unit's first dV/dK can start.
+            auto write_dkdv = [&]() -> bool {
+                if (!warp_wait(&sm.bar_dkdv_full, n & 1, ac)) return false;
+                tc_fence_after();
+                const int key = w.k0 + r;
+                const bool store = key < p.T;
+                const size_t off = ((size_t)w.bh * p.T + (store ? key : 0)) * D;
+#pragma unroll 1
+                for (int which = 0; which < 2; ++which) {
+                    __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + off;
+                    const uint32_t col0 = which == 0 ? C::kColDV : C::kColDK;
+                    const float mul = which == 0 ? 1.f : p.scale;     // dK = scale * dS^T Q
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t rr[32];
+                        tmem_ld32(t_lane + col0 + c * 32, rr);
+                        tmem_wait_ld();
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2)
+                            pk[e >> 1] = pack_bf16x2(__uint_as_float(rr[e]) * mul, __uint_as_float(rr[e + 1]) * mul);
+                        if (store) {
+                            uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+                            for (int v4 = 0; v4 < 4; ++v4)
+                                d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.bar_dkdv_free);
+                return true;
+            };
             for (int i = 0; i < w.n_q; ++i, ++g) {
+                const int b = g & 1;
                 if (!warp_wait(&sm.bar_dq_full, g & 1, ac)) { ok = false; break; }
                 tc_fence_after();
+                if (i == w.n_q - 1 && !(ok = __all_sync(0xffffffffu, write_dkdv()))) break;
                 uint32_t rr[64];
                 tmem_ld32(t_lane + C::kColDQ, *reinterpret_cast<uint32_t(*)[32]>(&rr[0]));
                 tmem_ld32(t_lane + C::kColDQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&rr[32]));
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&sm.bar_dq_free);
-                // Add dQ(g) into the fp32 accumulator: 32 columns at a time through the 16 KB staging
-                // buffer and a TMA bulk reduce-add of whole 128-byte rows (rows past T are skipped).
-                const uint32_t row_a = smem_u32(sm.dq_stage) + r * 128;
+                // Add dQ(g) into the fp32 accumulator: stage it in dS buffer b (dK(g) and dQ(g), the
+                // buffer's readers, completed before dq_full fired), two 32-column 128B-swizzled boxes,
+                // then two TMA bulk reduce-adds of whole 128-byte rows (rows past T are skipped).
+                const uint32_t stage = smem_u32(sm.ds[b]);
+#pragma unroll
                 for (int hq = 0; hq < 2; ++hq) {
-                    const int use = 2 * g + hq;             // uses of the staging buffer so far
-                    if (use > 0 && !warp_wait(&sm.bar_stage_free, (use - 1) & 1, ac)) { ok = false; break; }
+                    const uint32_t row_a = stage + hq * 16384 + r * 128;
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
                         st_shared_v4(row_a + ((c ^ (r & 7)) << 4), rr[hq * 32 + 4 * c], rr[hq * 32 + 4 * c + 1],
                                      rr[hq * 32 + 4 * c + 2], rr[hq * 32 + 4 * c + 3]);
-                    fence_proxy_async_smem();
-                    mbar_arrive(&sm.bar_stage_full);
-                    if (warp == 12 && lane == 0) {
-                        if (!mbar_wait(&sm.bar_stage_full, use & 1, ac)) { ok = false; break; }
-                        tma_reduce_add_3d(&tm_dq, sm.dq_stage, hq * 32, (w.qt_lo + i) * kTile, w.bh);
-                        bulk_commit_group();
-                        bulk_wait_group_read0();
-                        mbar_arrive(&sm.bar_stage_free);
-                    }
                 }
-                if (!ok) break;
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.bar_stage_full);
+                if (warp == 12 && lane == 0) {
+                    if (!mbar_wait(&sm.bar_stage_full, g & 1, ac)) { ok = false; break; }
+                    tma_reduce_add_3d(&tm_dq, sm.ds[b], 0, (w.qt_lo + i) * kTile, w.bh);
+                    tma_reduce_add_3d(&tm_dq, sm.ds[b] + 16384, 32, (w.qt_lo + i) * kTile, w.bh);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
+                    mbar_arrive(&sm.bar_ds_empty[b]);        // dS(g + 2) may be written now
+                }
             }
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
-            // ---------------------------------------------------------- dK / dV of this unit (thread = key row)
-            if (!warp_wait(&sm.bar_dkdv_full, n & 1, ac)) { ok = false; break; }
-            tc_fence_after();
-            const int key = w.k0 + r;
-            const bool store = key < p.T;
-            const size_t off = ((size_t)w.bh * p.T + (store ? key : 0)) * D;
-#pragma unroll 1
-            for (int which = 0; which < 2; ++which) {
-                __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + off;
-                const uint32_t col0 = which == 0 ? C::kColDV : C::kColDK;
-                const float mul = which == 0 ? 1.f : p.scale;     // dK = scale * dS^T Q
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t rr[32];
-                    tmem_ld32(t_lane + col0 + c * 32, rr);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2)
-                        pk[e >> 1] = pack_bf16x2(__uint_as_float(rr[e]) * mul, __uint_as_float(rr[e + 1]) * mul);
-                    if (store) {
-                        uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
-#pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4)
-                            d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-                    }
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(&sm.bar_dkdv_free);
         }
         if (warp == 12 && lane == 0) bulk_wait_group0();   // every reduce has landed in global memory
     }
