@@ -325,56 +325,78 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (!warp_wait(&sm.bar_s_full, g & 1, ac)) { ok = false; break; }
                 if (!warp_wait(&sm.bar_dp_full, g & 1, ac)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t rs[64], rd[64];
-                tmem_ld32(t_lane + C::kColS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
-                tmem_ld32(t_lane + C::kColS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
-                tmem_ld32(t_lane + C::kColDP + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&rd[0]));
-                tmem_ld32(t_lane + C::kColDP + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rd[32]));
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(&sm.bar_sdp_free);             // S^T, dP^T columns may be overwritten now
-
-                // Blocked (key, query) pairs get score -inf, hence P = 0 and dS = 0 exactly.  Done as
-                // a separate pass so the arithmetic loop below stays one branch-free block.
+                // The 64 query columns of this warpgroup are processed as two 32-column halves in a
+                // loop that is not unrolled (half the code of an unrolled pass); the second half's
+                // S^T and dP^T are read from TMEM while the first half is computed.
                 const bool need_mask = (qt == w.kt) || (W > 0 && qt * kTile + kTile - 1 >= w.k0 + W);
-                if (need_mask) {
-                    // Query columns that see this key form one range [c_lo, c_hi] (query >= key, and
-                    // query < key + W under a window): an unsigned compare and a select per element.
-                    const int c_lo = key - qc0;
-                    const int c_hi = W > 0 ? key + W - 1 - qc0 : INT_MAX / 2;
-                    const uint32_t span = (uint32_t)(c_hi - c_lo);
+                // Query columns that see this key form one range [c_lo, c_hi] (query >= key, and
+                // query < key + W under a window): blocked pairs get score -inf, hence P = dS = 0.
+                const int c_lo = key - qc0;
+                const int c_hi = W > 0 ? key + W - 1 - qc0 : INT_MAX / 2;
+                const uint32_t span = (uint32_t)(c_hi - c_lo);
+                const uint32_t row_a = smem_u32(sm.ds[b]) + h * 16384 + r * 128;
+                uint32_t xs[32], xd[32];
+                tmem_ld32(t_lane + C::kColS + h * 64, xs);
+                tmem_ld32(t_lane + C::kColDP + h * 64, xd);
+                tmem_wait_ld_regs2(xs, xd);
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    if (need_mask) {
 #pragma unroll
-                    for (int e = 0; e < 64; ++e)
-                        rs[e] = ((uint32_t)(e - c_lo) <= span) ? rs[e] : 0xff800000u;   // -inf
-                }
-                const float2* lse2 = reinterpret_cast<const float2*>(sm.lse2[s] + h * 64);
-                const float2* dlt = reinterpret_cast<const float2*>(sm.delta[s] + h * 64);
-                uint32_t pk[32], dk[32];
+                        for (int e = 0; e < 32; ++e)
+                            xs[e] = ((uint32_t)(hh * 32 + e - c_lo) <= span) ? xs[e] : 0xff800000u;   // -inf
+                    }
+                    const float4* lse4 = reinterpret_cast<const float4*>(sm.lse2[s] + h * 64 + hh * 32);
+                    const float4* dl4 = reinterpret_cast<const float4*>(sm.delta[s] + h * 64 + hh * 32);
+                    uint32_t pk[16], dk[16];
 #pragma unroll
-                for (int e = 0; e < 64; e += 2) {
-                    const float2 ls = lse2[e >> 1];
-                    const float2 dl = dlt[e >> 1];
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(rs[e]), sl2, -ls.x));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(rs[e + 1]), sl2, -ls.y));
-                    const float d0 = p0 * (__uint_as_float(rd[e]) - dl.x);
-                    const float d1 = p1 * (__uint_as_float(rd[e + 1]) - dl.y);
-                    pk[e >> 1] = pack_bf16x2(p0, p1);
-                    dk[e >> 1] = pack_bf16x2(d0, d1);
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 ls = lse4[e >> 2];
+                        const float4 dl = dl4[e >> 2];
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(xs[e]), sl2, -ls.x));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(xs[e + 1]), sl2, -ls.y));
+                        const float p2 = ex2_approx(fmaf(__uint_as_float(xs[e + 2]), sl2, -ls.z));
+                        const float p3 = ex2_approx(fmaf(__uint_as_float(xs[e + 3]), sl2, -ls.w));
+                        const float d0 = p0 * (__uint_as_float(xd[e]) - dl.x);
+                        const float d1 = p1 * (__uint_as_float(xd[e + 1]) - dl.y);
+                        const float d2 = p2 * (__uint_as_float(xd[e + 2]) - dl.z);
+                        const float d3 = p3 * (__uint_as_float(xd[e + 3]) - dl.w);
+                        pk[e >> 1] = pack_bf16x2(p0, p1);
+                        pk[(e >> 1) + 1] = pack_bf16x2(p2, p3);
+                        dk[e >> 1] = pack_bf16x2(d0, d1);
+                        dk[(e >> 1) + 1] = pack_bf16x2(d2, d3);
+                    }
+                    if (hh == 0) {
+                        // second half in flight while the first half is stored
+                        tmem_ld32(t_lane + C::kColS + h * 64 + 32, xs);
+                        tmem_ld32(t_lane + C::kColDP + h * 64 + 32, xd);
+                        // P^T(g) may go into TMEM once dV(g-1) has finished reading P^T(g-1); dS^T(g)
+                        // into shared buffer b once dK(g-2), dQ(g-2) have finished with it.
+                        if ((g > 0 && !warp_wait(&sm.bar_dv_done, (g - 1) & 1, ac)) ||
+                            (g >= 2 && !warp_wait(&sm.bar_ds_empty[b], ((g >> 1) - 1) & 1, ac))) {
+                            tmem_wait_ld();                // no load may be left in flight
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    tmem_st16(t_lane + C::kColP + h * 32 + hh * 16, pk);
+                    // Row r of half h holds queries [64h, 64h + 64): 8 chunks of 16 bytes, swizzled by row.
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int ch = hh * 4 + c;
+                        st_shared_v4(row_a + ((ch ^ (r & 7)) << 4), dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
+                    }
+                    if (hh == 0) {
+                        tmem_wait_ld_regs2(xs, xd);
+                        tc_fence_before();
+                        mbar_arrive(&sm.bar_sdp_free);     // S^T, dP^T columns may be overwritten now
+                    }
                 }
-                // P^T(g) into TMEM once dV(g-1) has finished reading P^T(g-1)
-                if (g > 0 && !warp_wait(&sm.bar_dv_done, (g - 1) & 1, ac)) { ok = false; break; }
-                tc_fence_after();
-                tmem_st32(t_lane + C::kColP + h * 32, pk);
+                if (!ok) break;
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.bar_p_full);
-                // dS^T(g) into shared buffer b once dK(g-2), dQ(g-2) have finished with it.
-                // Row r of half h holds queries [64h, 64h + 64): 8 chunks of 16 bytes, swizzled by row.
-                if (g >= 2 && !warp_wait(&sm.bar_ds_empty[b], ((g >> 1) - 1) & 1, ac)) { ok = false; break; }
-                const uint32_t row_a = smem_u32(sm.ds[b]) + h * 16384 + r * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    st_shared_v4(row_a + ((c ^ (r & 7)) << 4), dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3]);
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.bar_ds_full[b]);
             }
