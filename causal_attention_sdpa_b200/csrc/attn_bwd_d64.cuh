@@ -233,12 +233,12 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         tc_fence_after();
                         const uint32_t q_addr = smem_u32(sm.q[s]);
                         const uint32_t do_addr = smem_u32(sm.dout[s]);
-#pragma unroll
+#pragma unroll 1
                         for (int kk = 0; kk < D / 16; ++kk)
                             mma_ss(tmem + C::kColS, sw128_desc(k_addr + kk * 32, 16, 1024),
                                    sw128_desc(q_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
                         mma_commit(&sm.bar_s_full);
-#pragma unroll
+#pragma unroll 1
                         for (int kk = 0; kk < D / 16; ++kk)
                             mma_ss(tmem + C::kColDP, sw128_desc(v_addr + kk * 32, 16, 1024),
                                    sw128_desc(do_addr + kk * 32, 16, 1024), kIdescSS, kk > 0);
@@ -254,7 +254,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         if (i == 0 && n > 0 && !(ok = mbar_wait(&sm.bar_dkdv_free, (n - 1) & 1, ac))) break;
                         tc_fence_after();
                         const uint32_t do_addr = smem_u32(sm.dout[s]);
-#pragma unroll
+#pragma unroll 1
                         for (int kk = 0; kk < kTile / 16; ++kk)
                             mma_ts(tmem + C::kColDV, tmem + C::kColP + kk * 8,
                                    sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdescKxMN,
@@ -273,7 +273,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         tc_fence_after();
                         const uint32_t q_addr = smem_u32(sm.q[s]);
                         const uint32_t ds_addr = smem_u32(sm.ds[b]);
-#pragma unroll
+#pragma unroll 1
                         for (int kk = 0; kk < kTile / 16; ++kk) {
                             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
                             mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
@@ -283,7 +283,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         mma_commit(&sm.bar_qdo_empty[s]);
                         if (g > 0 && !(ok = mbar_wait(&sm.bar_dq_free, (g - 1) & 1, ac))) break;
                         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                         for (int kk = 0; kk < kTile / 16; ++kk)
                             mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
                                    sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
@@ -427,7 +427,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + off;
                     const uint32_t col0 = which == 0 ? C::kColDV : C::kColDK;
                     const float mul = which == 0 ? 1.f : p.scale;     // dK = scale * dS^T Q
-#pragma unroll
+#pragma unroll 1
                     for (int c = 0; c < 2; ++c) {
                         uint32_t rr[32];
                         tmem_ld32(t_lane + col0 + c * 32, rr);
