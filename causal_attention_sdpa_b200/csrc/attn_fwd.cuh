@@ -6,8 +6,15 @@
 // running max m and running sum l, rescaling the old sum by e^(m_old - m_new)
 // when the max grows).  The mapping onto sm_100a is this file's own:
 //
-//   one CTA = one (batch*head, 256-query block) = two 128-row Q tiles sharing
-//   every K/V tile it loads; 12 warps:
+//   one work item = one (batch*head, 256-query block) = two 128-row Q tiles sharing
+//   every K/V tile it loads.  The kernel is persistent: each CTA (one per SM, as
+//   TMEM allows) runs a fixed sequence of items, and every barrier phase counts
+//   tiles over all the items a role has handled, so the next item's Q load and
+//   first scores overlap the current item's last tiles and epilogue.  Items go
+//   out in waves of whole heads (the 256-query blocks of a head run at the same
+//   time, so its K/V tiles come from HBM once and from L2 to the other blocks);
+//   from one wave to the next, the block length class each CTA gets rotates, so
+//   every CTA gets an even mix of long and short blocks.  12 warps:
 //     warp 0       TMA producer: Q0, Q1 once, then K_j / V_j through a ring
 //     warp 1       TMEM allocator; issues S0 = Q0 K_j^T and S1 = Q1 K_j^T
 //     warps 2, 3   issue O0 += P0 V_j and O1 += P1 V_j (one MMA stream per warp)
@@ -48,14 +55,28 @@ struct FwdParams {
     int BH;
     int n_tiles;          // ceil(T / 128)
     int n_blocks;         // ceil(n_tiles / 2): 256-query blocks per head
+    int heads_per_wave;   // the grid is heads_per_wave * n_blocks CTAs
+    int n_waves;          // ceil(BH / heads_per_wave)
     int window;           // <= 0: causal only
     float scale_log2;     // scale * log2(e)
     uint64_t timeout_ns;
 };
 
+// Work item of CTA `cta` in wave `k`: head bh (or -1 when the wave has no item for it) and
+// 256-query block qb.  Slot s of a wave holds block class s / heads_per_wave (longest first)
+// of head s % heads_per_wave; a CTA's slot moves on by heads_per_wave each wave.
+__device__ __forceinline__ void fwd_item(const FwdParams& p, int cta, int k, int& bh, int& qb) {
+    const int G = p.heads_per_wave * p.n_blocks;
+    const int slot = (int)(((long long)cta + (long long)p.heads_per_wave * k) % G);
+    bh = p.heads_per_wave * k + slot % p.heads_per_wave;
+    qb = p.n_blocks - 1 - slot / p.heads_per_wave;
+    if (bh >= p.BH) bh = -1;
+}
+
 template <int D>
 struct FwdCfg {
     static constexpr int kStages = (D == 64) ? 3 : 2;
+    static constexpr int kQBufs = (D == 64) ? 2 : 1;   // items whose Q tiles can be resident at once
     static constexpr int kTileBytes = kTile * D * 2;
     static constexpr bool kSeparateP = (D == 64);
     static constexpr uint32_t kColS0 = 0, kColS1 = 128;
@@ -66,10 +87,11 @@ struct FwdCfg {
 template <int D>
 struct FwdSmem {
     using C = FwdCfg<D>;
-    alignas(1024) uint8_t q[2][C::kTileBytes];
+    alignas(1024) uint8_t q[C::kQBufs][2][C::kTileBytes];
     alignas(1024) uint8_t k[C::kStages][C::kTileBytes];
     alignas(1024) uint8_t v[C::kStages][C::kTileBytes];
-    uint64_t bar_q;
+    uint64_t bar_q[C::kQBufs];
+    uint64_t bar_q_empty[C::kQBufs];  // every S MMA of the item using this Q buffer finished
     uint64_t bar_k[C::kStages];
     uint64_t bar_v[C::kStages];
     uint64_t bar_kv_empty[C::kStages];
@@ -77,6 +99,7 @@ struct FwdSmem {
     uint64_t bar_s_free[2];
     uint64_t bar_p_full[2];
     uint64_t bar_o_done[2];
+    uint64_t bar_o_free[2];       // softmax warpgroup t has read its item's O out of TMEM
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -98,16 +121,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// (a, b) * s - m on the packed fp32x2 pipe.
-__device__ __forceinline__ void fma2_scale_sub(float& a, float& b, float s, float m) {
-    uint64_t x, sc, mm;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a), "f"(b));
-    asm("mov.b64 %0, {%1, %1};" : "=l"(sc) : "f"(s));
-    asm("mov.b64 %0, {%1, %1};" : "=l"(mm) : "f"(-m));
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(x) : "l"(x), "l"(sc), "l"(mm));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(x));
-}
-
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -117,6 +130,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(smem_align1024(smem_raw));
 
     constexpr int kStages = C::kStages;
+    constexpr int kQBufs = C::kQBufs;
     constexpr int kTileBytes = C::kTileBytes;
     constexpr int kBoxes = D / 64;                 // 64-column TMA boxes per tile
     constexpr uint32_t kTmemCols = 512;
@@ -125,18 +139,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // Blocks of one head are adjacent in launch order, so a head's K/V tiles are
-    // read from HBM once and then served from L2 to its other query blocks;
-    // within a head the longest blocks launch first.
-    const int bh = blockIdx.x / p.n_blocks;
-    const int qb = p.n_blocks - 1 - blockIdx.x % p.n_blocks;
-    int lo0, hi0, lo1, hi1;
-    fwd_key_range(2 * qb, p.window, lo0, hi0);
-    fwd_key_range(2 * qb + 1, p.window, lo1, hi1);
-    const int j_begin = lo0, j_end = hi1;
+    const int cta = blockIdx.x;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sm.bar_q, 1);
+        for (int b = 0; b < kQBufs; ++b) {
+            mbar_init(&sm.bar_q[b], 1);
+            mbar_init(&sm.bar_q_empty[b], 1);         // S warp
+        }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.bar_k[s], 1);
             mbar_init(&sm.bar_v[s], 1);
@@ -147,6 +156,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&sm.bar_s_free[t], 128);
             mbar_init(&sm.bar_p_full[t], 128);
             mbar_init(&sm.bar_o_done[t], 1);
+            mbar_init(&sm.bar_o_free[t], 128);
         }
         mbar_init(&sm.bar_drain, 3);
         sm.abort_flag = 0;
@@ -175,24 +185,41 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            mbar_arrive_expect_tx(&sm.bar_q, 2 * kTileBytes);
-            for (int t = 0; t < 2; ++t)
-                for (int b = 0; b < kBoxes; ++b)
-                    tma_load_3d(sm.q[t] + b * 16384, &tm_q, &sm.bar_q, b * 64, (2 * qb + t) * kTile, bh);
-            int it = 0;
-            for (int j = j_begin; j <= j_end; ++j, ++it) {
-                const int s = it % kStages;
-                const int n = it / kStages;
-                if (n > 0 && !mbar_wait(&sm.bar_kv_empty[s], (n - 1) & 1, ac)) break;
-                mbar_arrive_expect_tx(&sm.bar_k[s], kTileBytes);
-                for (int b = 0; b < kBoxes; ++b)
-                    tma_load_3d(sm.k[s] + b * 16384, &tm_k, &sm.bar_k[s], b * 64, j * kTile, bh);
-                mbar_arrive_expect_tx(&sm.bar_v[s], kTileBytes);
-                for (int b = 0; b < kBoxes; ++b)
-                    tma_load_3d(sm.v[s] + b * 16384, &tm_v, &sm.bar_v[s], b * 64, j * kTile, bh);
+            int it = 0;              // K/V tiles loaded, over all items
+            int n_item = 0;          // items whose Q was loaded
+            bool ok = true;
+            for (int k = 0; ok && k < p.n_waves; ++k) {
+                int bh, qb;
+                fwd_item(p, cta, k, bh, qb);
+                if (bh < 0) continue;
+                int lo0, hi0, lo1, hi1;
+                fwd_key_range(2 * qb, p.window, lo0, hi0);
+                fwd_key_range(2 * qb + 1, p.window, lo1, hi1);
+                const int qbuf = n_item % kQBufs;
+                if (n_item >= kQBufs &&
+                    !(ok = mbar_wait(&sm.bar_q_empty[qbuf], ((n_item / kQBufs) - 1) & 1, ac)))
+                    break;
+                mbar_arrive_expect_tx(&sm.bar_q[qbuf], 2 * kTileBytes);
+                for (int t = 0; t < 2; ++t)
+                    for (int b = 0; b < kBoxes; ++b)
+                        tma_load_3d(sm.q[qbuf][t] + b * 16384, &tm_q, &sm.bar_q[qbuf], b * 64, (2 * qb + t) * kTile, bh);
+                ++n_item;
+                for (int j = lo0; j <= hi1; ++j, ++it) {
+                    const int s = it % kStages;
+                    const int n = it / kStages;
+                    if (n > 0 && !(ok = mbar_wait(&sm.bar_kv_empty[s], (n - 1) & 1, ac))) break;
+                    mbar_arrive_expect_tx(&sm.bar_k[s], kTileBytes);
+                    for (int b = 0; b < kBoxes; ++b)
+                        tma_load_3d(sm.k[s] + b * 16384, &tm_k, &sm.bar_k[s], b * 64, j * kTile, bh);
+                    mbar_arrive_expect_tx(&sm.bar_v[s], kTileBytes);
+                    for (int b = 0; b < kBoxes; ++b)
+                        tma_load_3d(sm.v[s] + b * 16384, &tm_v, &sm.bar_v[s], b * 64, j * kTile, bh);
+                }
             }
             if (sm.abort_flag) {
-                mbar_wait_drain(&sm.bar_q, 0, p.timeout_ns);
+                // Let every load already issued land before the CTA exits.
+                for (int r = (n_item > kQBufs ? n_item - kQBufs : 0); r < n_item; ++r)
+                    mbar_wait_drain(&sm.bar_q[r % kQBufs], (r / kQBufs) & 1, p.timeout_ns);
                 for (int r = (it > kStages ? it - kStages : 0); r < it; ++r) {
                     mbar_wait_drain(&sm.bar_k[r % kStages], (r / kStages) & 1, p.timeout_ns);
                     mbar_wait_drain(&sm.bar_v[r % kStages], (r / kStages) & 1, p.timeout_ns);
@@ -206,60 +233,85 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         //   warp 1: S0 = Q0 K_j^T and S1 = Q1 K_j^T
         //   warp 2: O0 += P0 V_j        warp 3: O1 += P1 V_j
         // Each of the three warps releases a K/V stage once its own MMAs on it are done.
-        auto active = [&](int j, int t) { return t ? (j >= lo1 && j <= hi1) : (j >= lo0 && j <= hi0); };
         bool ok = true;
+        int it = 0;                  // K/V tiles consumed, over all items
+        int n_item = 0;
         if (warp == 1) {
-            const uint32_t q_addr0 = smem_u32(sm.q[0]), q_addr1 = smem_u32(sm.q[1]);
-            ok = mbar_wait(&sm.bar_q, 0, ac);
-            for (int j = j_begin; ok && j <= j_end; ++j) {
-                const int it = j - j_begin;
-                const int s = it % kStages;
-                if (!(ok = mbar_wait(&sm.bar_k[s], (it / kStages) & 1, ac))) break;
-                const uint32_t k_addr = smem_u32(sm.k[s]);
-                for (int t = 0; ok && t < 2; ++t) {
-                    if (!active(j, t)) continue;
-                    const int i = j - (t ? lo1 : lo0);
-                    if (i > 0) {
-                        // S_t shares TMEM with what the previous round still needs: the softmax copy of
-                        // S (separate P) or, when P is written over S, the PV MMA that reads it.
-                        uint64_t* freed = C::kSeparateP ? &sm.bar_s_free[t] : &sm.bar_o_done[t];
-                        if (!(ok = mbar_wait(freed, (i - 1) & 1, ac))) break;
-                    }
-                    tc_fence_after();
-                    const uint32_t q_addr = t ? q_addr1 : q_addr0;
-                    const uint32_t col = t ? C::kColS1 : C::kColS0;
+            int ct[2] = {0, 0};      // S tiles issued per warpgroup, over all items
+            for (int k = 0; ok && k < p.n_waves; ++k) {
+                int bh, qb;
+                fwd_item(p, cta, k, bh, qb);
+                if (bh < 0) continue;
+                int lo[2], hi[2];
+                fwd_key_range(2 * qb, p.window, lo[0], hi[0]);
+                fwd_key_range(2 * qb + 1, p.window, lo[1], hi[1]);
+                const int qbuf = n_item % kQBufs;
+                if (!(ok = mbar_wait(&sm.bar_q[qbuf], (n_item / kQBufs) & 1, ac))) break;
+                const uint32_t q_addr0 = smem_u32(sm.q[qbuf][0]), q_addr1 = smem_u32(sm.q[qbuf][1]);
+                for (int j = lo[0]; ok && j <= hi[1]; ++j, ++it) {
+                    const int s = it % kStages;
+                    if (!(ok = mbar_wait(&sm.bar_k[s], (it / kStages) & 1, ac))) break;
+                    const uint32_t k_addr = smem_u32(sm.k[s]);
+                    for (int t = 0; ok && t < 2; ++t) {
+                        if (j < lo[t] || j > hi[t]) continue;
+                        if (ct[t] > 0) {
+                            // S_t shares TMEM with what the previous tile still needs: the softmax
+                            // copy of S (separate P) or, when P is written over S, the PV MMA that reads it.
+                            uint64_t* freed = C::kSeparateP ? &sm.bar_s_free[t] : &sm.bar_o_done[t];
+                            if (!(ok = mbar_wait(freed, (ct[t] - 1) & 1, ac))) break;
+                        }
+                        tc_fence_after();
+                        const uint32_t q_addr = t ? q_addr1 : q_addr0;
+                        const uint32_t col = t ? C::kColS1 : C::kColS0;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        mma_ss(tmem + col, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
-                               kIdescQK, kk > 0);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                            mma_ss(tmem + col, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
+                                   kIdescQK, kk > 0);
+                        }
+                        mma_commit(&sm.bar_s_full[t]);
+                        ++ct[t];
                     }
-                    mma_commit(&sm.bar_s_full[t]);
+                    if (ok) mma_commit(&sm.bar_kv_empty[s]);
                 }
-                if (ok) mma_commit(&sm.bar_kv_empty[s]);
+                if (ok) mma_commit(&sm.bar_q_empty[qbuf]);    // the item's Q buffer may be reloaded
+                ++n_item;
             }
         } else if (warp == 2 || warp == 3) {
             const int t = warp - 2;
             const uint32_t col_o = t ? C::kColO1 : C::kColO0;
             const uint32_t col_p = t ? C::kColP1 : C::kColP0;
-            for (int j = j_begin; ok && j <= j_end; ++j) {
-                const int it = j - j_begin;
-                const int s = it % kStages;
-                if (!active(j, t)) {
-                    mbar_arrive(&sm.bar_kv_empty[s]);   // nothing of this warp reads stage s here
-                    continue;
-                }
-                const int i = j - (t ? lo1 : lo0);
-                if (!(ok = mbar_wait(&sm.bar_v[s], (it / kStages) & 1, ac))) break;
-                if (!(ok = mbar_wait(&sm.bar_p_full[t], i & 1, ac))) break;
-                tc_fence_after();
-                const uint32_t v_addr = smem_u32(sm.v[s]);
+            int ct = 0;              // PV tiles issued, over all items
+            for (int k = 0; ok && k < p.n_waves; ++k) {
+                int bh, qb;
+                fwd_item(p, cta, k, bh, qb);
+                if (bh < 0) continue;
+                int lo0, hi0, lo1, hi1;
+                fwd_key_range(2 * qb, p.window, lo0, hi0);
+                fwd_key_range(2 * qb + 1, p.window, lo1, hi1);
+                const int lo = t ? lo1 : lo0, hi = t ? hi1 : hi0;
+                for (int j = lo0; ok && j <= hi1; ++j, ++it) {
+                    const int s = it % kStages;
+                    if (j < lo || j > hi) {
+                        mbar_arrive(&sm.bar_kv_empty[s]);   // nothing of this warp reads stage s here
+                        continue;
+                    }
+                    const int i = j - lo;
+                    if (!(ok = mbar_wait(&sm.bar_v[s], (it / kStages) & 1, ac))) break;
+                    if (!(ok = mbar_wait(&sm.bar_p_full[t], ct & 1, ac))) break;
+                    // The item's first PV overwrites O: the previous item's epilogue must have read it.
+                    if (i == 0 && n_item > 0 && !(ok = mbar_wait(&sm.bar_o_free[t], (n_item - 1) & 1, ac))) break;
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_u32(sm.v[s]);
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ts(tmem + col_o, tmem + col_p + kk * 8, sw128_desc(v_addr + kk * 2048, 16384, 1024),
-                           kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&sm.bar_o_done[t]);
-                mma_commit(&sm.bar_kv_empty[s]);
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_ts(tmem + col_o, tmem + col_p + kk * 8, sw128_desc(v_addr + kk * 2048, 16384, 1024),
+                               kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&sm.bar_o_done[t]);
+                    mma_commit(&sm.bar_kv_empty[s]);
+                    ++ct;
+                }
+                ++n_item;
             }
         }
         if (warp <= 3) {
@@ -274,161 +326,173 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int t = (warp - 4) >> 2;               // Q tile of this warpgroup
         const int wq = warp & 3;                     // TMEM lane quarter this warp may access
         const int row = wq * 32 + lane;
-        const int qt = 2 * qb + t;
-        const int i_abs = qt * kTile + row;
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
         const uint32_t col_s = t ? C::kColS1 : C::kColS0;
         const uint32_t col_p = t ? C::kColP1 : C::kColP0;
         const uint32_t col_o = t ? C::kColO1 : C::kColO0;
         const float sl2 = p.scale_log2;
         const int W = p.window;
-        const int lo = t ? lo1 : lo0, hi = t ? hi1 : hi0;
-        float m_used = -INFINITY;    // reference max of the exponentials (log2 units)
-        float l = 0.f;               // running sum of 2^(x - m_used)
         bool ok = true;
-        const int n_t = hi - lo + 1;
-        for (int i = 0; i < n_t; ++i) {
-            const int j = lo + i;
-            const int k0 = j * kTile;
-            if (!warp_wait(&sm.bar_s_full[t], i & 1, ac)) { ok = false; break; }
-            tc_fence_after();
-            float s[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r[32];
-                tmem_ld32(t_lane + col_s + c * 32, r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
-            }
-            tmem_wait_ld();
-            if (C::kSeparateP) {
-                tc_fence_before();
-                mbar_arrive(&sm.bar_s_free[t]);        // S columns may be overwritten now
-            }
-            const bool need_mask = (j == qt) || (W > 0 && k0 <= qt * kTile + kTile - 1 - W);
-            if (need_mask) {
-                // Visible columns of this row form one range [c_lo, c_hi]; one unsigned compare
-                // and a select per element, no per-element branch.
-                const int c_hi = i_abs - k0;
-                const int c_lo = W > 0 ? i_abs - W + 1 - k0 : INT_MIN / 2;
-                const uint32_t span = (uint32_t)(c_hi - c_lo);
-#pragma unroll
-                for (int e = 0; e < 128; ++e)
-                    s[e] = ((uint32_t)(e - c_lo) <= span) ? s[e] : -INFINITY;
-            }
-            // Exponentials.  After the first tile of a row the reference max m_used is finite and
-            // the exponentials start at once with it, the tile's own max being computed in the
-            // same pass.  Only if some row's max now exceeds m_used by more than the lazy-rescale
-            // margin (rare) is the tile redone below with the new max; nothing has been stored or
-            // accumulated at that point.
-            uint32_t pk[64];
-            float rs = 0.f;
-            float mx;
-            if (i == 0) {
-                // First tile of this warpgroup: its max becomes the reference (O is still empty).
-                float m0 = fmax3(s[0], s[1], s[2]), m1 = fmax3(s[3], s[4], s[5]);
-                float m2 = fmax3(s[6], s[7], s[8]), m3 = fmax3(s[9], s[10], s[11]);
-#pragma unroll
-                for (int e = 12; e < 120; e += 8) {
-                    m0 = fmax3(m0, s[e], s[e + 1]);
-                    m1 = fmax3(m1, s[e + 2], s[e + 3]);
-                    m2 = fmax3(m2, s[e + 4], s[e + 5]);
-                    m3 = fmax3(m3, s[e + 6], s[e + 7]);
-                }
-                m0 = fmax3(m0, s[124], s[125]);
-                m1 = fmax3(m1, s[126], s[127]);
-                m2 = fmax3(m2, s[120], s[121]);
-                m3 = fmax3(m3, s[122], s[123]);
-                m_used = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;
-            }
-            {
-                const float m_spec = (m_used == -INFINITY) ? 0.f : m_used;
-                float m0 = -INFINITY, m1 = -INFINITY;
-                float r0 = 0.f, r1 = 0.f;
-#pragma unroll
-                for (int e = 0; e < 128; e += 4) {
-                    m0 = fmax3(m0, s[e], s[e + 1]);
-                    m1 = fmax3(m1, s[e + 2], s[e + 3]);
-                    const float a = ex2_approx(fmaf(s[e], sl2, -m_spec));
-                    const float b = ex2_approx(fmaf(s[e + 1], sl2, -m_spec));
-                    const float c = ex2_approx(fmaf(s[e + 2], sl2, -m_spec));
-                    const float d = ex2_approx(fmaf(s[e + 3], sl2, -m_spec));
-                    r0 += a + b;
-                    r1 += c + d;
-                    pk[e >> 1] = pack_bf16x2(a, b);
-                    pk[(e >> 1) + 1] = pack_bf16x2(c, d);
-                }
-                mx = fmaxf(m0, m1);
-                rs = r0 + r1;
-            }
-            const float m_new = mx * sl2;               // -inf stays -inf (sl2 > 0)
-            const bool need = m_new > m_used + kLazyRescale;
-            if (__any_sync(0xffffffffu, need)) {
-                const float alpha = need ? ex2_approx(m_used - m_new) : 1.f;
-                if (need) m_used = m_new;
-                l *= alpha;
-                if (i > 0) {
-                    // O holds PV up to tile i-1: wait for it, then rescale in place.
-                    if (!warp_wait(&sm.bar_o_done[t], (i - 1) & 1, ac)) { ok = false; break; }
-                    tc_fence_after();
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(t_lane + col_o + c * 32, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                        tmem_st32(t_lane + col_o + c * 32, r);
-                    }
-                }
-                // Redo this tile's exponentials against the new reference (rows that kept their
-                // reference recompute the same values).
-                const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
-                float r0 = 0.f, r1 = 0.f;
-#pragma unroll
-                for (int e = 0; e < 128; e += 2) {
-                    const float a = ex2_approx(fmaf(s[e], sl2, -m_use));
-                    const float b = ex2_approx(fmaf(s[e + 1], sl2, -m_use));
-                    r0 += a;
-                    r1 += b;
-                    pk[e >> 1] = pack_bf16x2(a, b);
-                }
-                rs = r0 + r1;
-            }
-            l += rs;
-            // Separate P columns: the previous PV must have finished reading them.
-            if (C::kSeparateP && i > 0) {
-                if (!warp_wait(&sm.bar_o_done[t], (i - 1) & 1, ac)) { ok = false; break; }
+        int ct = 0;                  // tiles of this warpgroup, over all items
+        for (int k = 0; ok && k < p.n_waves; ++k) {
+            int bh, qb;
+            fwd_item(p, cta, k, bh, qb);
+            if (bh < 0) continue;
+            const int qt = 2 * qb + t;
+            const int i_abs = qt * kTile + row;
+            int lo, hi;
+            fwd_key_range(qt, p.window, lo, hi);
+            float m_used = -INFINITY;    // reference max of the exponentials (log2 units)
+            float l = 0.f;               // running sum of 2^(x - m_used)
+            const int n_t = hi - lo + 1;
+            for (int i = 0; i < n_t; ++i) {
+                const int c = ct + i;    // phase index of this tile
+                const int j = lo + i;
+                const int k0 = j * kTile;
+                if (!warp_wait(&sm.bar_s_full[t], c & 1, ac)) { ok = false; break; }
                 tc_fence_after();
+                float s[128];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld32(t_lane + col_s + cc * 32, r);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) s[cc * 32 + e] = __uint_as_float(r[e]);
+                }
+                tmem_wait_ld();
+                if (C::kSeparateP) {
+                    tc_fence_before();
+                    mbar_arrive(&sm.bar_s_free[t]);        // S columns may be overwritten now
+                }
+                const bool need_mask = (j == qt) || (W > 0 && k0 <= qt * kTile + kTile - 1 - W);
+                if (need_mask) {
+                    // Visible columns of this row form one range [c_lo, c_hi]; one unsigned compare
+                    // and a select per element, no per-element branch.
+                    const int c_hi = i_abs - k0;
+                    const int c_lo = W > 0 ? i_abs - W + 1 - k0 : INT_MIN / 2;
+                    const uint32_t span = (uint32_t)(c_hi - c_lo);
+#pragma unroll
+                    for (int e = 0; e < 128; ++e)
+                        s[e] = ((uint32_t)(e - c_lo) <= span) ? s[e] : -INFINITY;
+                }
+                // Exponentials.  After the first tile of a row the reference max m_used is finite and
+                // the exponentials start at once with it, the tile's own max being computed in the
+                // same pass.  Only if some row's max now exceeds m_used by more than the lazy-rescale
+                // margin (rare) is the tile redone below with the new max; nothing has been stored or
+                // accumulated at that point.
+                uint32_t pk[64];
+                float rs = 0.f;
+                float mx;
+                if (i == 0) {
+                    // First tile of this item: its max becomes the reference (O is still empty).
+                    float m0 = fmax3(s[0], s[1], s[2]), m1 = fmax3(s[3], s[4], s[5]);
+                    float m2 = fmax3(s[6], s[7], s[8]), m3 = fmax3(s[9], s[10], s[11]);
+#pragma unroll
+                    for (int e = 12; e < 120; e += 8) {
+                        m0 = fmax3(m0, s[e], s[e + 1]);
+                        m1 = fmax3(m1, s[e + 2], s[e + 3]);
+                        m2 = fmax3(m2, s[e + 4], s[e + 5]);
+                        m3 = fmax3(m3, s[e + 6], s[e + 7]);
+                    }
+                    m0 = fmax3(m0, s[124], s[125]);
+                    m1 = fmax3(m1, s[126], s[127]);
+                    m2 = fmax3(m2, s[120], s[121]);
+                    m3 = fmax3(m3, s[122], s[123]);
+                    m_used = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;
+                }
+                {
+                    const float m_spec = (m_used == -INFINITY) ? 0.f : m_used;
+                    float m0 = -INFINITY, m1 = -INFINITY;
+                    float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 128; e += 4) {
+                        m0 = fmax3(m0, s[e], s[e + 1]);
+                        m1 = fmax3(m1, s[e + 2], s[e + 3]);
+                        const float a = ex2_approx(fmaf(s[e], sl2, -m_spec));
+                        const float b = ex2_approx(fmaf(s[e + 1], sl2, -m_spec));
+                        const float cx = ex2_approx(fmaf(s[e + 2], sl2, -m_spec));
+                        const float d = ex2_approx(fmaf(s[e + 3], sl2, -m_spec));
+                        r0 += a + b;
+                        r1 += cx + d;
+                        pk[e >> 1] = pack_bf16x2(a, b);
+                        pk[(e >> 1) + 1] = pack_bf16x2(cx, d);
+                    }
+                    mx = fmaxf(m0, m1);
+                    rs = r0 + r1;
+                }
+                const float m_new = mx * sl2;               // -inf stays -inf (sl2 > 0)
+                const bool need = m_new > m_used + kLazyRescale;
+                if (__any_sync(0xffffffffu, need)) {
+                    const float alpha = need ? ex2_approx(m_used - m_new) : 1.f;
+                    if (need) m_used = m_new;
+                    l *= alpha;
+                    if (i > 0) {
+                        // O holds PV up to the previous tile: wait for it, then rescale in place.
+                        if (!warp_wait(&sm.bar_o_done[t], (c - 1) & 1, ac)) { ok = false; break; }
+                        tc_fence_after();
+#pragma unroll
+                        for (int cc = 0; cc < D / 32; ++cc) {
+                            uint32_t r[32];
+                            tmem_ld32(t_lane + col_o + cc * 32, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                            tmem_st32(t_lane + col_o + cc * 32, r);
+                        }
+                    }
+                    // Redo this tile's exponentials against the new reference (rows that kept their
+                    // reference recompute the same values).
+                    const float m_use = (m_used == -INFINITY) ? 0.f : m_used;
+                    float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 128; e += 2) {
+                        const float a = ex2_approx(fmaf(s[e], sl2, -m_use));
+                        const float b = ex2_approx(fmaf(s[e + 1], sl2, -m_use));
+                        r0 += a;
+                        r1 += b;
+                        pk[e >> 1] = pack_bf16x2(a, b);
+                    }
+                    rs = r0 + r1;
+                }
+                l += rs;
+                // Separate P columns: the previous PV (possibly the previous item's last) must have
+                // finished reading them.
+                if (C::kSeparateP && c > 0) {
+                    if (!warp_wait(&sm.bar_o_done[t], (c - 1) & 1, ac)) { ok = false; break; }
+                    tc_fence_after();
+                }
+                tmem_st32(t_lane + col_p, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+                tmem_st32(t_lane + col_p + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sm.bar_p_full[t]);
             }
-            tmem_st32(t_lane + col_p, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(t_lane + col_p + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&sm.bar_p_full[t]);
-        }
-        // ---------------------------------------------------------- epilogue
-        if (__all_sync(0xffffffffu, ok) && warp_wait(&sm.bar_o_done[t], (n_t - 1) & 1, ac)) {
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            ct += n_t;
+            // ------------------------------------------------------ epilogue of this item
+            if (!warp_wait(&sm.bar_o_done[t], (ct - 1) & 1, ac)) { ok = false; break; }
             tc_fence_after();
             const float inv_l = 1.f / l;
             const bool store = i_abs < p.T;
             __nv_bfloat16* orow = p.o + ((size_t)bh * p.T + (store ? i_abs : 0)) * D;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t r[32];
-                tmem_ld32(t_lane + col_o + c * 32, r);
+                tmem_ld32(t_lane + col_o + cc * 32, r);
                 tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2)
                     pk[e >> 1] = pack_bf16x2(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
                 if (store) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+                    uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4)
                         dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&sm.bar_o_free[t]);               // O columns may be overwritten now
             if (store) p.lse[(size_t)bh * p.T + i_abs] = (m_used + log2f(l)) * 0.69314718055994531f;
         }
     }

@@ -99,6 +99,8 @@ bool set_smem(Kern k, size_t bytes) {
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
 }
 
+int sm_count();
+
 template <int D>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH, int T, float scale,
                int window, cudaStream_t st) {
@@ -115,9 +117,19 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.window = window > 0 ? window : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = wait_timeout_ns();
+    // D = 64: persistent grid, waves of whole heads, heads_per_wave * n_blocks CTAs, at most one
+    // per SM (TMEM holds one CTA's accumulators) unless a single head has more blocks than the GPU
+    // has SMs.  D = 128: one item per CTA (a single wave of all heads): its Q tiles cannot be
+    // double-buffered next to the K/V ring, so a CTA would wait for each new item's Q.
+    const int sms = sm_count();
+    int hpw = D == 64 ? sms / p.n_blocks : BH;
+    if (hpw < 1) hpw = 1;
+    if (hpw > BH) hpw = BH;
+    p.heads_per_wave = hpw;
+    p.n_waves = (BH + hpw - 1) / hpw;
     const size_t smem = sizeof(FwdSmem<D>) + 1024;
     if (!set_smem(attn_fwd_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
-    const unsigned grid = (unsigned)((long long)p.n_blocks * BH);
+    const unsigned grid = (unsigned)((long long)hpw * p.n_blocks);
     attn_fwd_kernel<D><<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
