@@ -41,8 +41,7 @@ constexpr int kBwd64Threads = 512;
 
 struct Bwd64Cfg {
     static constexpr int D = 64;
-    static constexpr int kQStages = 3;                       // Q (+ lse2) ring depth
-    static constexpr int kDoStages = 2;                      // dO (+ Delta) ring depth
+    static constexpr int kStages = 2;                        // Q/dO ring depth
     static constexpr int kTileBytes = kTile * D * 2;         // 16 KB
     static constexpr uint32_t kColS = 0, kColDP = 128, kColP = 256, kColDV = 320, kColDK = 384, kColDQ = 448;
     // Threads that read each unit id: warps 1..3 (one lane each) + 256 P/dS + 128 dQ.
@@ -53,22 +52,20 @@ struct Bwd64Smem {
     using C = Bwd64Cfg;
     alignas(1024) uint8_t k[2][C::kTileBytes];
     alignas(1024) uint8_t v[2][C::kTileBytes];
-    alignas(1024) uint8_t q[C::kQStages][C::kTileBytes];
-    alignas(1024) uint8_t dout[C::kDoStages][C::kTileBytes];
+    alignas(1024) uint8_t q[C::kStages][C::kTileBytes];
+    alignas(1024) uint8_t dout[C::kStages][C::kTileBytes];
     // dS^T bf16 [key][query] as two 64-query halves; once dK(g) and dQ(g) have read it, the same
     // 32 KB stages dQ(g) in fp32 as two [128 rows][32 cols] 128B-swizzled boxes for the reduce.
     alignas(1024) uint8_t ds[2][kTile * kTile * 2];
-    alignas(16) float lse2[C::kQStages][kTile];
-    alignas(16) float delta[C::kDoStages][kTile];
+    alignas(16) float lse2[C::kStages][kTile];
+    alignas(16) float delta[C::kStages][kTile];
     int unit[2];                  // work-unit ring: id, or -1 when there is no more work
     uint64_t bar_unit_full[2];
     uint64_t bar_unit_empty[2];
     uint64_t bar_kv_full[2];
     uint64_t bar_kv_empty[2];     // S/dP warp and dK/dQ warp done with this K/V buffer
-    uint64_t bar_q_full[C::kQStages];
-    uint64_t bar_q_empty[C::kQStages];       // dK(g) finished reading Q(g)
-    uint64_t bar_do_full[C::kDoStages];
-    uint64_t bar_do_empty[C::kDoStages];     // dV(g) finished reading dO(g)
+    uint64_t bar_qdo_full[C::kStages];
+    uint64_t bar_qdo_empty[C::kStages];
     uint64_t bar_s_full;
     uint64_t bar_dp_full;
     uint64_t bar_sdp_free;        // both P/dS warpgroups have S(g), dP(g) in registers
@@ -109,8 +106,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     Bwd64Smem& sm = *reinterpret_cast<Bwd64Smem*>(smem_align1024(smem_raw));
 
-    constexpr int kQStages = C::kQStages;
-    constexpr int kDoStages = C::kDoStages;
+    constexpr int kStages = C::kStages;
     constexpr int kTileBytes = C::kTileBytes;
     constexpr uint32_t kTmemCols = 512;
     constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);    // S^T = K Q^T, dP^T = V dO^T
@@ -130,13 +126,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&sm.bar_ds_full[b], 256);
             mbar_init(&sm.bar_ds_empty[b], 1);      // by the dQ reduce issuer
         }
-        for (int s = 0; s < kQStages; ++s) {
-            mbar_init(&sm.bar_q_full[s], 1);
-            mbar_init(&sm.bar_q_empty[s], 1);       // by the dK warp's commit
-        }
-        for (int s = 0; s < kDoStages; ++s) {
-            mbar_init(&sm.bar_do_full[s], 1);
-            mbar_init(&sm.bar_do_empty[s], 1);      // by the dV warp's commit
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.bar_qdo_full[s], 1);
+            mbar_init(&sm.bar_qdo_empty[s], 2);     // dV warp + dK warp
         }
         mbar_init(&sm.bar_s_full, 1);
         mbar_init(&sm.bar_dp_full, 1);
@@ -183,8 +175,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_do);
-            int g = 0;                         // query tiles whose Q was loaded
-            int g_issued_do = 0;               // query tiles whose dO was loaded
+            int g = 0;                         // query tiles loaded so far
             int n_kv = 0;                      // K/V buffers loaded so far
             bool ok = true;
             for (int n = 0; ok; ++n) {
@@ -203,29 +194,24 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tma_load_3d(sm.v[kb], &tm_v, &sm.bar_kv_full[kb], 0, w.k0, w.bh);
                 n_kv = n + 1;
                 for (int i = 0; i < w.n_q; ++i, ++g) {
+                    const int s = g % kStages;
+                    const int m = g / kStages;
+                    if (m > 0 && !(ok = mbar_wait(&sm.bar_qdo_empty[s], (m - 1) & 1, ac))) break;
                     const int q0 = (w.qt_lo + i) * kTile;
+                    mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + 2 * kTile * 4);
+                    tma_load_3d(sm.q[s], &tm_q, &sm.bar_qdo_full[s], 0, q0, w.bh);
+                    tma_load_3d(sm.dout[s], &tm_do, &sm.bar_qdo_full[s], 0, q0, w.bh);
                     const size_t roff = (size_t)w.bh * p.T_pad + q0;
-                    const int sq = g % kQStages, mq = g / kQStages;
-                    if (mq > 0 && !(ok = mbar_wait(&sm.bar_q_empty[sq], (mq - 1) & 1, ac))) break;
-                    mbar_arrive_expect_tx(&sm.bar_q_full[sq], kTileBytes + kTile * 4);
-                    tma_load_3d(sm.q[sq], &tm_q, &sm.bar_q_full[sq], 0, q0, w.bh);
-                    bulk_load(sm.lse2[sq], p.lse2 + roff, kTile * 4, &sm.bar_q_full[sq]);
-                    const int sd = g % kDoStages, md = g / kDoStages;
-                    if (md > 0 && !(ok = mbar_wait(&sm.bar_do_empty[sd], (md - 1) & 1, ac))) { ++g; break; }
-                    mbar_arrive_expect_tx(&sm.bar_do_full[sd], kTileBytes + kTile * 4);
-                    tma_load_3d(sm.dout[sd], &tm_do, &sm.bar_do_full[sd], 0, q0, w.bh);
-                    bulk_load(sm.delta[sd], p.delta + roff, kTile * 4, &sm.bar_do_full[sd]);
-                    g_issued_do = g + 1;
+                    bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
+                    bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_qdo_full[s]);
                 }
             }
             if (sm.abort_flag) {
                 // Let every load already issued land before the CTA exits.
                 for (int r = (n_kv > 2 ? n_kv - 2 : 0); r < n_kv; ++r)
                     mbar_wait_drain(&sm.bar_kv_full[r & 1], (r >> 1) & 1, p.timeout_ns);
-                for (int r = (g > kQStages ? g - kQStages : 0); r < g; ++r)
-                    mbar_wait_drain(&sm.bar_q_full[r % kQStages], (r / kQStages) & 1, p.timeout_ns);
-                for (int r = (g_issued_do > kDoStages ? g_issued_do - kDoStages : 0); r < g_issued_do; ++r)
-                    mbar_wait_drain(&sm.bar_do_full[r % kDoStages], (r / kDoStages) & 1, p.timeout_ns);
+                for (int r = (g > kStages ? g - kStages : 0); r < g; ++r)
+                    mbar_wait_drain(&sm.bar_qdo_full[r % kStages], (r / kStages) & 1, p.timeout_ns);
             }
         } else if (lane == 0 && warp >= 1) {
             // -------------------------------------------------------- MMA issuers
@@ -241,13 +227,12 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (warp == 1) {
                     if (!(ok = mbar_wait(&sm.bar_kv_full[kb], (n >> 1) & 1, ac))) break;
                     for (int i = 0; i < w.n_q; ++i, ++g) {
-                        const int sq = g % kQStages, sd = g % kDoStages;
-                        if (!(ok = mbar_wait(&sm.bar_q_full[sq], (g / kQStages) & 1, ac))) break;
-                        if (!(ok = mbar_wait(&sm.bar_do_full[sd], (g / kDoStages) & 1, ac))) break;
+                        const int s = g % kStages;
+                        if (!(ok = mbar_wait(&sm.bar_qdo_full[s], (g / kStages) & 1, ac))) break;
                         if (g > 0 && !(ok = mbar_wait(&sm.bar_sdp_free, (g - 1) & 1, ac))) break;
                         tc_fence_after();
-                        const uint32_t q_addr = smem_u32(sm.q[sq]);
-                        const uint32_t do_addr = smem_u32(sm.dout[sd]);
+                        const uint32_t q_addr = smem_u32(sm.q[s]);
+                        const uint32_t do_addr = smem_u32(sm.dout[s]);
 #pragma unroll 1
                         for (int kk = 0; kk < D / 16; ++kk)
                             mma_ss(tmem + C::kColS, sw128_desc(k_addr + kk * 32, 16, 1024),
@@ -264,7 +249,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     // dV += P^T dO; the first one of a unit overwrites dV once the previous
                     // unit's dV has been copied out.
                     for (int i = 0; i < w.n_q; ++i, ++g) {
-                        const int s = g % kDoStages;
+                        const int s = g % kStages;
                         if (!(ok = mbar_wait(&sm.bar_p_full, g & 1, ac))) break;
                         if (i == 0 && n > 0 && !(ok = mbar_wait(&sm.bar_dkdv_free, (n - 1) & 1, ac))) break;
                         tc_fence_after();
@@ -275,13 +260,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                    sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdescKxMN,
                                    (i > 0 || kk > 0) ? 1u : 0u);
                         mma_commit(&sm.bar_dv_done);
-                        mma_commit(&sm.bar_do_empty[s]);
+                        mma_commit(&sm.bar_qdo_empty[s]);
                     }
                     if (ok) mma_commit(&sm.bar_dkdv_full);
                 } else if (warp == 3) {
                     // dK += dS^T Q, then dQ = dS K once the dQ warpgroup has copied out dQ(g-1)
                     for (int i = 0; i < w.n_q; ++i, ++g) {
-                        const int s = g % kQStages;
+                        const int s = g % kStages;
                         const int b = g & 1;
                         if (!(ok = mbar_wait(&sm.bar_ds_full[b], (g >> 1) & 1, ac))) break;
                         if (i == 0 && n > 0 && !(ok = mbar_wait(&sm.bar_dkdv_free, (n - 1) & 1, ac))) break;
@@ -295,7 +280,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                    sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN,
                                    (i > 0 || kk > 0) ? 1u : 0u);
                         }
-                        mma_commit(&sm.bar_q_empty[s]);
+                        mma_commit(&sm.bar_qdo_empty[s]);
                         if (g > 0 && !(ok = mbar_wait(&sm.bar_dq_free, (g - 1) & 1, ac))) break;
                         tc_fence_after();
 #pragma unroll 1
@@ -332,12 +317,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const Bwd64Unit w = bwd64_unit(u, p);
             const int key = w.k0 + r;
             for (int i = 0; i < w.n_q; ++i, ++g) {
-                const int sq = g % kQStages, sd = g % kDoStages;
+                const int s = g % kStages;
                 const int b = g & 1;
                 const int qt = w.qt_lo + i;
                 const int qc0 = qt * kTile + h * 64;       // first query column of this half
-                if (!warp_wait(&sm.bar_q_full[sq], (g / kQStages) & 1, ac)) { ok = false; break; }
-                if (!warp_wait(&sm.bar_do_full[sd], (g / kDoStages) & 1, ac)) { ok = false; break; }
+                if (!warp_wait(&sm.bar_qdo_full[s], (g / kStages) & 1, ac)) { ok = false; break; }
                 if (!warp_wait(&sm.bar_s_full, g & 1, ac)) { ok = false; break; }
                 if (!warp_wait(&sm.bar_dp_full, g & 1, ac)) { ok = false; break; }
                 tc_fence_after();
@@ -362,8 +346,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         for (int e = 0; e < 32; ++e)
                             xs[e] = ((uint32_t)(hh * 32 + e - c_lo) <= span) ? xs[e] : 0xff800000u;   // -inf
                     }
-                    const float4* lse4 = reinterpret_cast<const float4*>(sm.lse2[sq] + h * 64 + hh * 32);
-                    const float4* dl4 = reinterpret_cast<const float4*>(sm.delta[sd] + h * 64 + hh * 32);
+                    const float4* lse4 = reinterpret_cast<const float4*>(sm.lse2[s] + h * 64 + hh * 32);
+                    const float4* dl4 = reinterpret_cast<const float4*>(sm.delta[s] + h * 64 + hh * 32);
                     uint32_t pk[16], dk[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 4) {
