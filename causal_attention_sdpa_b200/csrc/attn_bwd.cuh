@@ -92,14 +92,6 @@ struct BwdSmem {
     int abort_flag;
 };
 
-// Query tiles that see at least one key of key tile kt: [kt, qt_hi].
-__device__ __forceinline__ int bwd_last_query_tile(int kt, int n_tiles, int window) {
-    if (window <= 0) return n_tiles - 1;
-    const long last = (long)kt * kTile + kTile - 1 + window - 1;   // last query that sees a key of the tile
-    const long t = last / kTile;
-    return t < n_tiles - 1 ? (int)t : n_tiles - 1;
-}
-
 // Delta_i = dO_i . O_i, lse2_i = lse_i * log2(e) for every padded row, and a
 // zeroed fp32 dQ accumulator.  G = D / 8 threads per row, 16-byte accesses.
 // No thread leaves before the group shuffle (every lane of the warp takes part).

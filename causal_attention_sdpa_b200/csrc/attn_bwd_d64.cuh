@@ -89,11 +89,9 @@ struct Bwd64Unit {
 
 __device__ __forceinline__ Bwd64Unit bwd64_unit(int u, const BwdParams& p) {
     Bwd64Unit w;
-    w.bh = u / p.n_tiles;
-    w.kt = u % p.n_tiles;
+    bwd_unit(u, p.n_tiles, p.window, w.bh, w.kt, w.n_q);   // schedule.h
     w.k0 = w.kt * kTile;
     w.qt_lo = w.kt;
-    w.n_q = bwd_last_query_tile(w.kt, p.n_tiles, p.window) - w.qt_lo + 1;
     return w;
 }
 

@@ -40,11 +40,11 @@
 
 #include <climits>
 
+#include "schedule.h"
 #include "sm100.cuh"
 
 namespace gpt_attn {
 
-constexpr int kTile = 128;           // rows per Q tile and per K/V tile
 constexpr int kFwdThreads = 384;
 constexpr float kLazyRescale = 8.0f; // log2 units
 
@@ -62,15 +62,9 @@ struct FwdParams {
     uint64_t timeout_ns;
 };
 
-// Work item of CTA `cta` in wave `k`: head bh (or -1 when the wave has no item for it) and
-// 256-query block qb.  Slot s of a wave holds block class s / heads_per_wave (longest first)
-// of head s % heads_per_wave; a CTA's slot moves on by heads_per_wave each wave.
+// Work item of CTA `cta` in wave `k` (schedule.h).
 __device__ __forceinline__ void fwd_item(const FwdParams& p, int cta, int k, int& bh, int& qb) {
-    const int G = p.heads_per_wave * p.n_blocks;
-    const int slot = (int)(((long long)cta + (long long)p.heads_per_wave * k) % G);
-    bh = p.heads_per_wave * k + slot % p.heads_per_wave;
-    qb = p.n_blocks - 1 - slot / p.heads_per_wave;
-    if (bh >= p.BH) bh = -1;
+    fwd_item(p.heads_per_wave, p.n_blocks, p.BH, cta, k, bh, qb);
 }
 
 template <int D>
@@ -104,16 +98,6 @@ struct FwdSmem {
     uint32_t tmem_base;
     int abort_flag;
 };
-
-// Key tiles [lo, hi] hold every key visible to some query of Q tile qt.
-__device__ __forceinline__ void fwd_key_range(int qt, int window, int& lo, int& hi) {
-    hi = qt;
-    lo = 0;
-    if (window > 0) {
-        const int first = qt * kTile - window + 1;
-        lo = first > 0 ? first / kTile : 0;
-    }
-}
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;

@@ -121,12 +121,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     // per SM (TMEM holds one CTA's accumulators) unless a single head has more blocks than the GPU
     // has SMs.  D = 128: one item per CTA (a single wave of all heads): its Q tiles cannot be
     // double-buffered next to the K/V ring, so a CTA would wait for each new item's Q.
-    const int sms = sm_count();
-    int hpw = D == 64 ? sms / p.n_blocks : BH;
-    if (hpw < 1) hpw = 1;
-    if (hpw > BH) hpw = BH;
-    p.heads_per_wave = hpw;
-    p.n_waves = (BH + hpw - 1) / hpw;
+    fwd_grid(sm_count(), p.n_blocks, BH, D == 64, p.heads_per_wave, p.n_waves);
+    const int hpw = p.heads_per_wave;
     const size_t smem = sizeof(FwdSmem<D>) + 1024;
     if (!set_smem(attn_fwd_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
     const unsigned grid = (unsigned)((long long)hpw * p.n_blocks);
