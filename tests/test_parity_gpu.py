@@ -5,10 +5,10 @@ Tolerances (fixed for this path): max |dO| <= 2e-2 on O, <= 5e-2 on dQ/dK/dV,
 relative Frobenius error <= 1e-2 on each, and max |d lse| <= 1e-3.
 
 The five workloads run at full size on the GPU, in the launch configuration
-the benchmark times; the oracle checks every element of every head for the
-four T <= 1024 workloads and a spread of 6 sampled heads (first and last
-included) for the 8192-token sliding-window one.  Small odd shapes cover ragged tails, tiny T,
-windows and both head dimensions over all heads.
+the benchmark times, and the oracle checks every element of every head of all
+five (the 8192-token sliding-window one takes about a minute of fp64 on the host
+cores).  Small odd shapes cover ragged tails, tiny T, windows and both head
+dimensions over all heads.
 """
 import math
 
@@ -18,7 +18,7 @@ import torch
 
 import oracle
 import workloads
-from workloads import WORKLOADS, make_inputs, sample_heads
+from workloads import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -84,11 +84,9 @@ def compare(got, ref, heads=None, label=""):
 def test_workload_parity(ga, w):
     q, k, v, do = workloads.workload_inputs(w)
     got = run_gpu(ga, q, k, v, do, w.scale, w.window)
-    # every head of every tensor, except the 8192-token workload, where the fp64 oracle
-    # checks a spread of 6 of its 24 heads (first and last included)
-    heads = sample_heads(w.B, w.H, 6, seed=w.index) if w.T > 4096 else None
-    ref = run_oracle(q, k, v, do, w.scale, w.window, heads)
-    compare(got, ref, heads, label=f"cfg{w.index}")
+    # every element of every head of every output
+    ref = run_oracle(q, k, v, do, w.scale, w.window)
+    compare(got, ref, None, label=f"cfg{w.index}")
 
 
 ODD = [
