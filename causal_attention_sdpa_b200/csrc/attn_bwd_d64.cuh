@@ -16,7 +16,9 @@
 //     warps 8..11   P/dS warpgroup for query columns [64, 128)
 //     warps 12..15  dQ warpgroup: copies dQ(g) out of TMEM and adds it into the
 //                   fp32 accumulator (staged in the dS buffer dQ(g) has just read,
-//                   then TMA bulk reduce-add); writes each unit's dK (x scale) and dV
+//                   then TMA bulk reduce-add); writes each unit's dK (x scale) and dV,
+//                   staged in the unit's own K and V buffers (no MMA reads them any
+//                   more), with two TMA tile stores
 //   The MMAs are spread over three issuing warps: one thread cannot issue
 //   128-row MMAs of N <= 128 fast enough to keep the tensor pipe busy.
 //   TMEM (512 columns): S^T [0,128)  dP^T [128,256)  P^T bf16 [256,320)
@@ -63,7 +65,7 @@ struct Bwd64Smem {
     uint64_t bar_unit_full[2];
     uint64_t bar_unit_empty[2];
     uint64_t bar_kv_full[2];
-    uint64_t bar_kv_empty[2];     // S/dP warp and dK/dQ warp done with this K/V buffer
+    uint64_t bar_kv_empty[2];     // S/dP warp, dK/dQ warp and the dK/dV stores done with this K/V buffer
     uint64_t bar_qdo_full[C::kStages];
     uint64_t bar_qdo_empty[C::kStages];
     uint64_t bar_s_full;
@@ -78,6 +80,7 @@ struct Bwd64Smem {
     uint64_t bar_dkdv_full;       // last dV and dK of a unit finished
     uint64_t bar_dkdv_free;       // dK, dV of a unit copied out of TMEM
     uint64_t bar_stage_full;      // the dQ warpgroup has staged dQ(g)
+    uint64_t bar_dkdv_staged;     // the dQ warpgroup has staged a unit's dK and dV
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -98,7 +101,8 @@ __device__ __forceinline__ Bwd64Unit bwd64_unit(int u, const BwdParams& p) {
 __global__ void __launch_bounds__(kBwd64Threads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+                const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
+                const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
     using C = Bwd64Cfg;
     constexpr int D = C::D;
     extern __shared__ uint8_t smem_raw[];
@@ -120,7 +124,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&sm.bar_unit_full[b], 1);
             mbar_init(&sm.bar_unit_empty[b], C::kUnitReaders);
             mbar_init(&sm.bar_kv_full[b], 1);
-            mbar_init(&sm.bar_kv_empty[b], 2);
+            mbar_init(&sm.bar_kv_empty[b], 3);
             mbar_init(&sm.bar_ds_full[b], 256);
             mbar_init(&sm.bar_ds_empty[b], 1);      // by the dQ reduce issuer
         }
@@ -138,6 +142,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(&sm.bar_dkdv_full, 2);            // last dV + last dK of the unit
         mbar_init(&sm.bar_dkdv_free, 128);
         mbar_init(&sm.bar_stage_full, 128);
+        mbar_init(&sm.bar_dkdv_staged, 128);
         mbar_init(&sm.bar_drain, 3);                // the three MMA-issuing threads
         sm.abort_flag = 0;
         fence_barrier_init();
@@ -412,38 +417,50 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ok = __all_sync(0xffffffffu, read_unit(n, u));
             if (!ok || u < 0) break;
             const Bwd64Unit w = bwd64_unit(u, p);
-            // dK / dV of this unit (thread = key row): copied out as soon as the unit's last dQ is
-            // complete, before that dQ is reduced, so the next unit's first dV/dK can start.
+            const int kb = n & 1;
+            // dK / dV of this unit (thread = key row): copied out of TMEM as soon as the unit's last
+            // dQ is complete, before that dQ is reduced, so the next unit's first dV/dK can start.
+            // They are staged as bf16 128B-swizzled tiles in this unit's V and K buffers, which no
+            // MMA reads any more (the last dP and dQ of the unit completed before dkdv_full), and
+            // written with TMA tile stores (rows past T are clipped), so every warp writes whole
+            // lines.  The buffers go back to the producer once the stores have read them.
             auto write_dkdv = [&]() -> bool {
                 if (!warp_wait(&sm.bar_dkdv_full, n & 1, ac)) return false;
                 tc_fence_after();
-                const int key = w.k0 + r;
-                const bool store = key < p.T;
-                const size_t off = ((size_t)w.bh * p.T + (store ? key : 0)) * D;
 #pragma unroll 1
                 for (int which = 0; which < 2; ++which) {
-                    __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + off;
                     const uint32_t col0 = which == 0 ? C::kColDV : C::kColDK;
                     const float mul = which == 0 ? 1.f : p.scale;     // dK = scale * dS^T Q
+                    const uint32_t row_a = smem_u32(which == 0 ? sm.v[kb] : sm.k[kb]) + r * 128;
 #pragma unroll 1
                     for (int c = 0; c < 2; ++c) {
                         uint32_t rr[32];
                         tmem_ld32(t_lane + col0 + c * 32, rr);
                         tmem_wait_ld();
-                        uint32_t pk[16];
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2)
-                            pk[e >> 1] = pack_bf16x2(__uint_as_float(rr[e]) * mul, __uint_as_float(rr[e + 1]) * mul);
-                        if (store) {
-                            uint4* d4 = reinterpret_cast<uint4*>(dst_row + c * 32);
+                        for (int j = 0; j < 4; ++j) {
+                            uint32_t v4[4];
 #pragma unroll
-                            for (int v4 = 0; v4 < 4; ++v4)
-                                d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                            for (int e = 0; e < 4; ++e)
+                                v4[e] = pack_bf16x2(__uint_as_float(rr[8 * j + 2 * e]) * mul,
+                                                    __uint_as_float(rr[8 * j + 2 * e + 1]) * mul);
+                            const int chunk = c * 4 + j;             // 8 bf16 columns per 16-byte chunk
+                            st_shared_v4(row_a + ((chunk ^ (r & 7)) << 4), v4[0], v4[1], v4[2], v4[3]);
                         }
                     }
                 }
                 tc_fence_before();
                 mbar_arrive(&sm.bar_dkdv_free);
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.bar_dkdv_staged);
+                if (warp == 12 && lane == 0) {
+                    if (!mbar_wait(&sm.bar_dkdv_staged, n & 1, ac)) return false;
+                    tma_store_3d(&tm_dv, sm.v[kb], 0, w.k0, w.bh);
+                    tma_store_3d(&tm_dk, sm.k[kb], 0, w.k0, w.bh);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
+                    mbar_arrive(&sm.bar_kv_empty[kb]);
+                }
                 return true;
             };
             for (int i = 0; i < w.n_q; ++i, ++g) {

@@ -207,13 +207,15 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
     const long long units = (long long)w.n_tiles * BH;
     const unsigned grid = (unsigned)units;
     if constexpr (D == 64) {
-        CUtensorMap mdq;
-        if (!make_tmap_f32_acc(&mdq, w.dq_acc, BH, T, D)) return GPT_ATTN_ERR_CUDA;
+        CUtensorMap mdq, mdk, mdv;
+        if (!make_tmap_f32_acc(&mdq, w.dq_acc, BH, T, D) || !make_tmap_bf16(&mdk, dk, BH, T, D) ||
+            !make_tmap_bf16(&mdv, dv, BH, T, D))
+            return GPT_ATTN_ERR_CUDA;
         const size_t smem = sizeof(Bwd64Smem) + 1024;
         if (!set_smem(attn_bwd_kernel, smem)) return GPT_ATTN_ERR_CUDA;
         // persistent: one CTA per SM, work units taken from the counter in the workspace
         const unsigned pgrid = (unsigned)(units < sm_count() ? units : sm_count());
-        attn_bwd_kernel<<<pgrid, kBwd64Threads, smem, st>>>(mq, mk, mv, mdo, mdq, p);
+        attn_bwd_kernel<<<pgrid, kBwd64Threads, smem, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p);
     } else {
         const size_t smem = sizeof(BwdSmem<D>) + 1024;
         if (!set_smem(attn_bwd_serial_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
