@@ -73,6 +73,7 @@ struct FwdCfg {
     static constexpr int kQBufs = (D == 64) ? 2 : 1;   // items whose Q tiles can be resident at once
     static constexpr int kTileBytes = kTile * D * 2;
     static constexpr bool kSeparateP = (D == 64);
+    static constexpr bool kOStage = (D == 64);          // O tiles staged in shared memory for TMA stores
     static constexpr uint32_t kColS0 = 0, kColS1 = 128;
     static constexpr uint32_t kColP0 = kSeparateP ? 256u : 0u, kColP1 = kSeparateP ? 320u : 128u;
     static constexpr uint32_t kColO0 = kSeparateP ? 384u : 256u, kColO1 = kSeparateP ? 448u : 384u;
@@ -84,6 +85,7 @@ struct FwdSmem {
     alignas(1024) uint8_t q[C::kQBufs][2][C::kTileBytes];
     alignas(1024) uint8_t k[C::kStages][C::kTileBytes];
     alignas(1024) uint8_t v[C::kStages][C::kTileBytes];
+    alignas(1024) uint8_t ostage[C::kOStage ? 2 : 1][C::kOStage ? C::kTileBytes : 16];
     uint64_t bar_q[C::kQBufs];
     uint64_t bar_q_empty[C::kQBufs];  // every S MMA of the item using this Q buffer finished
     uint64_t bar_k[C::kStages];
@@ -94,6 +96,8 @@ struct FwdSmem {
     uint64_t bar_p_full[2];
     uint64_t bar_o_done[2];
     uint64_t bar_o_free[2];       // softmax warpgroup t has read its item's O out of TMEM
+    uint64_t bar_ostage_free[2];  // warpgroup t's previous O tile store has read its staging buffer
+    uint64_t bar_ostage_full[2];  // warpgroup t has staged its O tile
     uint64_t bar_drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -108,7 +112,8 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                const FwdParams p) {
     using C = FwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(smem_align1024(smem_raw));
@@ -141,6 +146,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&sm.bar_p_full[t], 128);
             mbar_init(&sm.bar_o_done[t], 1);
             mbar_init(&sm.bar_o_free[t], 128);
+            mbar_init(&sm.bar_ostage_free[t], 1);
+            mbar_init(&sm.bar_ostage_full[t], 128);
         }
         mbar_init(&sm.bar_drain, 3);
         sm.abort_flag = 0;
@@ -318,6 +325,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int W = p.window;
         bool ok = true;
         int ct = 0;                  // tiles of this warpgroup, over all items
+        int n_items = 0;
+        const bool o_issuer = wq == 0 && lane == 0;   // issues this warpgroup's O tile stores
         for (int k = 0; ok && k < p.n_waves; ++k) {
             int bh, qb;
             fwd_item(p, cta, k, bh, qb);
@@ -458,27 +467,69 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             const float inv_l = 1.f / l;
             const bool store = i_abs < p.T;
-            __nv_bfloat16* orow = p.o + ((size_t)bh * p.T + (store ? i_abs : 0)) * D;
-#pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t r[32];
-                tmem_ld32(t_lane + col_o + cc * 32, r);
-                tmem_wait_ld();
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2)
-                    pk[e >> 1] = pack_bf16x2(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
-                if (store) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            if constexpr (C::kOStage) {
+                // O is staged as a bf16 128B-swizzled tile and written with one TMA tile store (rows
+                // past T are clipped), so every warp writes whole lines; the staging buffer is
+                // reused once the previous item's store has read it.
+                if (o_issuer) {
+                    bulk_wait_group_read0();
+                    mbar_arrive(&sm.bar_ostage_free[t]);
                 }
+                if (!warp_wait(&sm.bar_ostage_free[t], n_items & 1, ac)) { ok = false; break; }
+                const uint32_t row_a = smem_u32(sm.ostage[t]) + row * 128;
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld32(t_lane + col_o + cc * 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j4 = 0; j4 < 4; ++j4) {
+                        uint32_t v4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            v4[e] = pack_bf16x2(__uint_as_float(r[8 * j4 + 2 * e]) * inv_l,
+                                                __uint_as_float(r[8 * j4 + 2 * e + 1]) * inv_l);
+                        const int chunk = cc * 4 + j4;           // 16-byte chunk of the 128-byte row
+                        st_shared_v4(row_a + ((chunk ^ (row & 7)) << 4), v4[0], v4[1], v4[2], v4[3]);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.bar_o_free[t]);           // O columns may be overwritten now
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.bar_ostage_full[t]);
+                if (o_issuer) {
+                    if (!mbar_wait(&sm.bar_ostage_full[t], n_items & 1, ac)) {
+                        ok = false;
+                    } else if (qt * kTile < p.T) {               // a tile wholly past T stores nothing
+                        tma_store_3d(&tm_o, sm.ostage[t], 0, qt * kTile, bh);
+                        bulk_commit_group();
+                    }
+                }
+            } else {
+                __nv_bfloat16* orow = p.o + ((size_t)bh * p.T + (store ? i_abs : 0)) * D;
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld32(t_lane + col_o + cc * 32, r);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2)
+                        pk[e >> 1] = pack_bf16x2(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
+                    if (store) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.bar_o_free[t]);           // O columns may be overwritten now
             }
-            tc_fence_before();
-            mbar_arrive(&sm.bar_o_free[t]);               // O columns may be overwritten now
+            ++n_items;
             if (store) p.lse[(size_t)bh * p.T + i_abs] = (m_used + log2f(l)) * 0.69314718055994531f;
         }
+        if (C::kOStage && o_issuer) bulk_wait_group0();   // the last O store has landed
     }
 
     tc_fence_before();

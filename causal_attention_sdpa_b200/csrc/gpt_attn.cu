@@ -104,8 +104,9 @@ int sm_count();
 template <int D>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH, int T, float scale,
                int window, cudaStream_t st) {
-    CUtensorMap mq, mk, mv;
-    if (!make_tmap_bf16(&mq, q, BH, T, D) || !make_tmap_bf16(&mk, k, BH, T, D) || !make_tmap_bf16(&mv, v, BH, T, D))
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_tmap_bf16(&mq, q, BH, T, D) || !make_tmap_bf16(&mk, k, BH, T, D) || !make_tmap_bf16(&mv, v, BH, T, D) ||
+        !make_tmap_bf16(&mo, o, BH, T, D))
         return GPT_ATTN_ERR_CUDA;
     FwdParams p;
     p.o = static_cast<__nv_bfloat16*>(o);
@@ -126,7 +127,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     const size_t smem = sizeof(FwdSmem<D>) + 1024;
     if (!set_smem(attn_fwd_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
     const unsigned grid = (unsigned)((long long)hpw * p.n_blocks);
-    attn_fwd_kernel<D><<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, p);
+    attn_fwd_kernel<D><<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, mo, p);
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
