@@ -83,8 +83,11 @@ size_t gpt_attn_bwd_workspace_bytes(int B, int H, int T, int D);
  *   workspace      : device buffer of at least gpt_attn_bwd_workspace_bytes(B,H,T,D)
  *                    bytes, 16-byte aligned, owned by the caller; its contents on
  *                    entry are ignored and on return are unspecified.
- * The dQ accumulation uses fp32 atomics, so dQ may differ between runs in the
- * last bits (summation order); dK, dV and the forward pass are deterministic.
+ * The dQ contributions of the key tiles are added into the fp32 accumulator by
+ * bulk reductions whose order varies between runs, so dQ may differ in the last
+ * bits; dK, dV and the forward pass are deterministic.  The workspace also holds
+ * the backward kernel's work-unit counter: backward calls whose work may overlap
+ * on the GPU need distinct workspaces.
  * Returns GPT_ATTN_OK or an error code.  Asynchronous on `stream`.
  */
 int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o,
