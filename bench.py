@@ -64,8 +64,9 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, units: float):
-    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+def recorded_traffic(kernel: str, w):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current kernel
+    source and on a workload of the same T, D and window (bytes scale with B*H)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
@@ -74,8 +75,9 @@ def recorded_traffic(kernel: str, units: float):
     e = d.get(kernel)
     if not e or e.get("source_hash") != kernel_source_hash():
         return None
-    # bytes were captured on e["units"] (b*h*T^2 pairs-equivalent units); scale to this launch
-    return e["dram_bytes"] * units / e["units"]
+    if (e.get("T"), e.get("D"), e.get("window")) != (w.T, w.D, w.window):
+        return None
+    return e["dram_bytes"] * (w.B * w.H) / e["units"]
 
 
 class ClockSampler:
@@ -328,7 +330,7 @@ def main():
                 "peak_source": f"{peaks['source']} burst dense bf16",
                 "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
                                       if peaks.get("bf16_tflops_sustained") else None),
-                "traffic": recorded_traffic(dominant, B * H)}
+                "traffic": recorded_traffic(dominant, w)}
     n_el = B * H * T * D
     prep_bytes = 2 * n_el * 2 + 4 * n_el + B * H * T * 4 * 3
     kernels = {n: {"ms": per_kernel[n]} for n in per_kernel}
