@@ -1,0 +1,54 @@
+"""Host logic of bench.py that needs no GPU: the flop counts behind the metric, the workload
+description, and when a recorded ncu DRAM-traffic figure may be reported."""
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench      # noqa: E402
+import workloads  # noqa: E402
+
+
+def test_flop_counts():
+    # causal: fwd 2*B*H*T^2*D, fwd+bwd 3.5x that (bwd 2.5x)
+    assert workloads.fwd_flops(64, 12, 1024, 64) == pytest.approx(2 * 64 * 12 * 1024 ** 2 * 64)
+    assert workloads.fwd_bwd_flops(64, 12, 1024, 64) == pytest.approx(7 * 64 * 12 * 1024 ** 2 * 64)
+    # windowed: 4*D per visible pair; T=8192, W=1024 has sum_i min(i+1, W) visible pairs per head
+    pairs = sum(min(i + 1, 1024) for i in range(8192))
+    assert workloads.fwd_flops(4, 6, 8192, 128, 1024) == pytest.approx(4 * 128 * pairs * 24)
+    assert workloads.fwd_bwd_flops(4, 6, 8192, 128, 1024) / 1e9 == pytest.approx(338.3, rel=1e-3)
+
+
+def test_l2_note_tells_resident_from_streamed_inputs():
+    assert "larger than L2" in bench.l2_note(workloads.BY_INDEX[3])
+    assert "fit in L2" in bench.l2_note(workloads.BY_INDEX[1])
+
+
+def test_workload_config_names_the_workload():
+    c = bench.workload_config(workloads.HEADLINE)
+    for key in ("workload", "B", "H", "T", "D", "window", "scale", "seed", "l2", "flop_count"):
+        assert key in c
+    assert c["workload"] and "model" not in c
+
+
+def test_recorded_traffic_is_gated_by_source_hash_and_shape(tmp_path, monkeypatch):
+    w3 = workloads.BY_INDEX[3]
+    rec = {"attn_bwd_kernel": {"source_hash": bench.kernel_source_hash(), "dram_bytes": 768e6, "units": 768,
+                               "T": w3.T, "D": w3.D, "window": w3.window}}
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: rec["attn_bwd_kernel"]["source_hash"])
+    assert bench.recorded_traffic("attn_bwd_kernel", w3) == pytest.approx(768e6)
+    # same T, D, window, fewer heads: scaled by B*H
+    assert bench.recorded_traffic("attn_bwd_kernel", workloads.BY_INDEX[2]) == pytest.approx(768e6 * 96 / 768)
+    # another shape, another kernel, or changed sources: nothing reported
+    assert bench.recorded_traffic("attn_bwd_kernel", workloads.BY_INDEX[5]) is None
+    assert bench.recorded_traffic("attn_fwd_kernel", w3) is None
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
+    assert bench.recorded_traffic("attn_bwd_kernel", w3) is None
+
