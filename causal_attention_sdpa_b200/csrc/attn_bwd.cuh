@@ -12,16 +12,19 @@
 //                          per-head rows of the workspace; zeroes the fp32 dQ
 //                          accumulator.  HBM-bound.
 //   attn_bwd_kernel (D=64, attn_bwd_d64.cuh) / attn_bwd_serial_kernel (D=128,
-//                          this file): one CTA per (batch*head, 128-key tile);
-//                          K and V stay in shared memory, query tiles stream
-//                          through a TMA ring.  Per query tile, five tcgen05 MMAs:
+//                          this file): per (batch*head, 128-key tile), K and V
+//                          stay in shared memory while the query tiles that see
+//                          them stream through a TMA ring (D=64: persistent CTAs
+//                          taking these units from a counter; D=128: one CTA per
+//                          unit).  Per query tile, five tcgen05 MMAs:
 //                            S^T  = K Q^T          (TMEM)
 //                            dP^T = V dO^T         (TMEM)
 //                            dV  += P^T dO         (P^T read from TMEM)
 //                            dK  += dS^T Q         (dS^T from shared memory)
 //                            dQ   = dS K           (same shared tile, MN-major)
-//                          dQ is added into the fp32 accumulator with vector
-//                          red.global.add by a dedicated warpgroup.
+//                          dQ is added into the fp32 accumulator by TMA bulk
+//                          reduce-adds (D=64) or vector red.global.add (D=128)
+//                          from a dedicated warpgroup.
 //   attn_dq_convert_kernel dQ = bf16(scale * fp32 accumulator).
 // dS is rounded to bf16 unscaled; the score scale is applied once per output
 // element, in the dK epilogue and in the dQ conversion.

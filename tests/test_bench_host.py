@@ -52,3 +52,18 @@ def test_recorded_traffic_is_gated_by_source_hash_and_shape(tmp_path, monkeypatc
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
     assert bench.recorded_traffic("attn_bwd_kernel", w3) is None
 
+
+
+def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    import shutil
+    src = os.path.join(ROOT, "causal_attention_sdpa_b200", "csrc")
+    dst = tmp_path / "causal_attention_sdpa_b200" / "csrc"
+    shutil.copytree(src, dst)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash()
+    f = dst / "schedule.h"
+    text = f.read_text()
+    f.write_text(text.replace("// Key tiles [lo, hi]", "// (reworded)  Key tiles [lo, hi]") + "\n/* note */\n")
+    assert bench.kernel_source_hash() == h0
+    f.write_text(text.replace("constexpr int kTile = 128;", "constexpr int kTile = 64;"))
+    assert bench.kernel_source_hash() != h0
