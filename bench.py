@@ -89,8 +89,74 @@ def recorded_traffic(kernel: str, w):
     return e["dram_bytes"] * (w.B * w.H) / e["units"]
 
 
+class NvmlClockSampler:
+    """SM clock and clock-event (throttle) reasons read through NVML about every 2 ms while
+    running, so that even a timed region of a few milliseconds is sampled from inside."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown", 0x8),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap", 0x4))
+
+    def __init__(self, device):
+        self.device = device
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
+        self._nvml = None
+
+    def __enter__(self):
+        try:
+            import threading
+
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            pr = torch.cuda.get_device_properties(self.device)
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(
+                "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id))
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._stop = threading.Event()
+
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                             pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                    except Exception:
+                        return
+                    self._stop.wait(0.002)
+
+            self._thread = threading.Thread(target=run, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._thread = None
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2.0)
+        if self._nvml is not None:
+            try:
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
+        return False
+
+    def summary(self):
+        if not self.samples:
+            return None
+        bits = {name: getattr(self._nvml, attr, default) for name, attr, default in self.REASONS}
+        reasons = sorted({name for _, r in self.samples for name, b in bits.items() if r & b})
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml, inside the timed region"}
+
+
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running (used when NVML
+    cannot be read)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
@@ -273,9 +339,10 @@ def main():
     with ClockSampler(local) as clk:
         time.sleep(0.25)   # let the sampler start before the timed region
         barrier()
-        for i in range(args.steps):
-            step(evs[i])
-        barrier()
+        with NvmlClockSampler(dev) as nclk:
+            for i in range(args.steps):
+                step(evs[i])
+            barrier()
     status = ga.gpt_attn_check(stream)
     if status != ga.GPT_ATTN_OK:
         raise RuntimeError(f"timed steps failed: {ga.status_string(status)}")
@@ -362,7 +429,7 @@ def main():
         "data": "synthetic", "config": workload_config(w),
         "pct_of_peak": value / world / peaks["bf16_tflops"],
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": 4 * args.steps, "clocks": clk.summary(),
+        "gpu_launches": 4 * args.steps, "clocks": nclk.summary() or clk.summary(),
     }
     print(json.dumps(line), flush=True)
     if dist is not None:
