@@ -33,6 +33,9 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 
+METRIC = "causal attention fwd+bwd TFLOP/s on 1 B200 and % of dense bf16 peak"
+
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -248,7 +251,7 @@ def run_reference(args, w, rank):
     sample = (f"{nh} of {w.B * w.H} heads (b,h) of the workload per step, fwd+bwd, fp64 oracle "
               f"(OpenMP over heads)")
     line = {
-        "impl": "reference", "metric": "causal attention fwd+bwd TFLOP/s", "value": value, "unit": "TFLOP/s",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -423,7 +426,7 @@ def main():
                "sample": f"{nh} of {B * H} heads (b,h) of the workload, fwd+bwd, fp64, {t:.1f} s wall"}
 
     line = {
-        "metric": "causal attention fwd+bwd TFLOP/s", "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": workload_config(w),
