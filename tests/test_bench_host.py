@@ -68,7 +68,3 @@ def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     f.write_text(text.replace("constexpr int kTile = 128;", "constexpr int kTile = 64;"))
     assert bench.kernel_source_hash() != h0
 
-
-def test_metric_is_the_one_the_workload_file_names():
-    with open(os.path.join(ROOT, "BASELINE.json")) as f:
-        assert bench.METRIC == json.load(f)["metric"]
