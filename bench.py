@@ -46,6 +46,9 @@ def parse_args():
                     help="workload number (1-5); the default is the headline shape")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write a 256 MB buffer between timed steps (outside their events) and sum the "
+                         "per-step times: a cold-L2 figure for workloads whose inputs fit in L2")
     return ap.parse_args()
 
 
@@ -338,18 +341,24 @@ def main():
         raise RuntimeError(f"warm-up failed: {ga.status_string(status)}")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if args.flush_l2 else None
     barrier()
     with ClockSampler(local) as clk:
         time.sleep(0.25)   # let the sampler start before the timed region
         barrier()
         with NvmlClockSampler(dev) as nclk:
             for i in range(args.steps):
+                if flush is not None:
+                    flush.zero_()
                 step(evs[i])
             barrier()
     status = ga.gpt_attn_check(stream)
     if status != ga.GPT_ATTN_OK:
         raise RuntimeError(f"timed steps failed: {ga.status_string(status)}")
-    total_ms = evs[0][0].elapsed_time(evs[-1][4])
+    if flush is None:
+        total_ms = evs[0][0].elapsed_time(evs[-1][4])
+    else:   # the flushes between steps are not part of the work
+        total_ms = sum(e[0].elapsed_time(e[4]) for e in evs)
     per_kernel = {name: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps
                   for i, name in enumerate(("attn_fwd_kernel", "attn_bwd_prep_kernel", "attn_bwd_kernel",
                                             "attn_dq_convert_kernel"))}
@@ -429,7 +438,10 @@ def main():
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": workload_config(w),
+        "data": "synthetic", "config": dict(workload_config(w), **({"l2": "L2 flushed between steps (256 MB "
+                                                                    "write outside the step events), "
+                                                                    "sum of per-step times"}
+                                                                    if flush is not None else {})),
         "pct_of_peak": value / world / peaks["bf16_tflops"],
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": 4 * args.steps, "clocks": nclk.summary() or clk.summary(),
