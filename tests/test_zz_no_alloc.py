@@ -6,8 +6,9 @@ or a process whose memory belongs to a pooling allocator).  For them the
 library offers gpt_attn_bwd_noalloc, which uses a fixed 32 MiB scratch array
 inside the library instead of a caller-supplied workspace.  These tests call
 it through the C ABI and check it against gpt_attn_bwd, which takes its
-workspace from the caller, on two calls in a row: the second call reuses
-the scratch the first one left behind, with a different shape.
+workspace from the caller, and against the fp64 CPU oracle, on two calls in
+a row: the second call reuses the scratch the first one left behind, with a
+different shape.
 
 This file is collected last on purpose, so a run that stops at the first
 failure has already run every other test.
@@ -20,6 +21,7 @@ import pytest
 import torch
 
 import causal_attention_sdpa_b200 as ga
+import oracle
 from workloads import make_inputs
 
 TOL_GRAD, TOL_FRO = 5e-2, 1e-2          # the gradient tolerances of the parity tests
@@ -35,7 +37,9 @@ def _noalloc(L, t, scale, window, stream):
 
 
 def _close(name, got, ref):
-    g, r = got.double(), ref.double()
+    g = got.double().cpu()
+    r = torch.as_tensor(np.asarray(ref, dtype=np.float64)) if not torch.is_tensor(ref) else ref.double().cpu()
+    r = r.reshape(g.shape)
     err = (g - r).abs().max().item()
     assert err <= TOL_GRAD, f"{name}: max |err| {err:.3e}"
     rn = r.norm().item()
@@ -52,21 +56,25 @@ def test_noalloc_matches_workspace_backward_on_two_calls():
     build.build()
     L = ga.lib()
     stream = torch.cuda.current_stream()
-    cases = [  # (B, H, T, D, window, scale, seed): the second is smaller and uses D = 128
-        (2, 3, 1000, 64, 0, 0.125, 11),
+    cases = [  # (B, H, T, D, window, scale, seed): the first runs several work units per CTA on a
+        # ragged T under a window; the second is smaller and uses D = 128
+        (2, 48, 1000, 64, 200, 0.125, 11),
         (1, 2, 777, 128, 333, 0.12, 12),
     ]
     for B, H, T, D, W, s, seed in cases:
-        q, k, v, do = (x.cuda() for x in make_inputs(B, H, T, D, seed=seed))
+        q_h, k_h, v_h, do_h = make_inputs(B, H, T, D, seed=seed)
+        q, k, v, do = (x.cuda() for x in (q_h, k_h, v_h, do_h))
         o, lse = ga.gpt_attn_fwd(q, k, v, scale=s, window=W)
         ref = ga.gpt_attn_bwd(q, k, v, o, lse, do, scale=s, window=W)
         got = [torch.full_like(q, float("nan")) for _ in range(3)]
         rc = _noalloc(L, [q, k, v, o, lse, do] + got, s, W, stream)
         assert rc == ga.GPT_ATTN_OK, ga.status_string(rc)
         assert ga.gpt_attn_check(stream) == ga.GPT_ATTN_OK
-        for name, g_, r_ in zip(("dq", "dk", "dv"), got, ref):
+        exact = oracle.attn_bwd(q_h, k_h, v_h, do_h, s, W)[:3]
+        for name, g_, r_, x_ in zip(("dq", "dk", "dv"), got, ref, exact):
             assert torch.isfinite(g_).all(), name
-            _close(f"B{B}H{H}T{T}D{D} {name}", g_, r_)
+            _close(f"B{B}H{H}T{T}D{D} {name} vs gpt_attn_bwd", g_, r_)
+            _close(f"B{B}H{H}T{T}D{D} {name} vs oracle", g_, x_)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
