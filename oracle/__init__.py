@@ -52,6 +52,13 @@ def _load():
         lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, L, L, L, ctypes.c_double, L,
                                         dp, dp, dp, dp, ctypes.c_int]
         lib.oracle_attn_bwd.restype = ctypes.c_int
+        lp = ctypes.POINTER(ctypes.c_long)
+        lib.oracle_attn_fwd_masked.argtypes = [dp, dp, dp, L, L, L, L, ctypes.c_double, lp, L, lp,
+                                               dp, dp, ctypes.c_int]
+        lib.oracle_attn_fwd_masked.restype = ctypes.c_int
+        lib.oracle_attn_bwd_masked.argtypes = [dp, dp, dp, dp, L, L, L, L, ctypes.c_double, lp, L, lp,
+                                               dp, dp, dp, dp, ctypes.c_int]
+        lib.oracle_attn_bwd_masked.restype = ctypes.c_int
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -105,3 +112,54 @@ def attn_bwd(q, k, v, dO, scale: float, window: int = 0, nthreads: int = 0):
         raise RuntimeError(f"oracle_attn_bwd failed with code {rc}")
     return dq, dk, dv, delta
 
+
+
+def _long_array(x, n=None):
+    if x is None:
+        return None, None
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.int64).reshape(-1)).astype(ctypes.c_long)
+    if n is not None and a.size != n:
+        raise ValueError(f"expected {n} entries, got {a.size}")
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_long))
+
+
+def attn_fwd_masked(q, k, v, scale: float, head_windows=None, window: int = 0, doc_start=None,
+                    nthreads: int = 0):
+    """Forward pass with a window per head and document boundaries.
+
+    q, k, v: [B, H, T, D].  head_windows: H ints (window of head h in every batch row) or None
+    for `window` everywhere.  doc_start: [B, T] ints, the first position of the document holding
+    each token, or None for one document per row.  Returns (O [B,H,T,D], lse [B,H,T]) in fp64."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    if not (q.shape == k.shape == v.shape) or q.ndim != 4:
+        raise ValueError("q, k, v must share one shape [B, H, T, D]")
+    B, H, T, D = q.shape
+    hw, hwp = _long_array(head_windows, H)
+    ds, dsp = _long_array(doc_start, B * T)
+    o = np.zeros_like(q)
+    lse = np.zeros((B, H, T), dtype=np.float64)
+    rc = _load().oracle_attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), B, H, T, D, float(scale), hwp,
+                                        int(window), dsp, _ptr(o), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_masked failed with code {rc}")
+    return o, lse
+
+
+def attn_bwd_masked(q, k, v, dO, scale: float, head_windows=None, window: int = 0, doc_start=None,
+                    nthreads: int = 0):
+    """Backward pass of sum(O * dO) under the mask of attn_fwd_masked.
+    Returns (dQ, dK, dV, Delta) in fp64."""
+    q, k, v, dO = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dO)
+    if not (q.shape == k.shape == v.shape == dO.shape) or q.ndim != 4:
+        raise ValueError("q, k, v, dO must share one shape [B, H, T, D]")
+    B, H, T, D = q.shape
+    hw, hwp = _long_array(head_windows, H)
+    ds, dsp = _long_array(doc_start, B * T)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    delta = np.zeros((B, H, T), dtype=np.float64)
+    rc = _load().oracle_attn_bwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), B, H, T, D, float(scale),
+                                        hwp, int(window), dsp, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(delta),
+                                        int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_bwd_masked failed with code {rc}")
+    return dq, dk, dv, delta

@@ -23,7 +23,10 @@
  *   the window is the sliding-window variant named in the modded-nanogpt
  *   README's technique list (long/short sliding-window attention).  Masked
  *   entries are -inf before the softmax, so every row renormalises over its
- *   visible keys.
+ *   visible keys.  The masked entry points add, from the same list, a window
+ *   per head (the long/short pattern) and document boundaries (batches
+ *   aligned to document ends): key j must also not lie before the start of
+ *   the document that holds token i.
  *
  *   Backward: the exact gradient of L = sum(O * dO) with respect to Q, K, V
  *   (the pages only call loss.backward(); the gradient of the definition
@@ -46,19 +49,25 @@
 #include <omp.h>
 #endif
 
-static int visible(long i, long j, long window) {
+/* Key j is visible to query i iff j <= i, (window <= 0 or j > i - window), and
+ * j >= first, the position where the document holding token i starts (0 when
+ * the sequence is one document).  The document rule is the reading taken of the
+ * modded-nanogpt README's item on aligning batches to document ends: attention
+ * stays inside a document. */
+static int visible(long i, long j, long window, long first) {
     if (j > i) return 0;
     if (window > 0 && j <= i - window) return 0;
+    if (j < first) return 0;
     return 1;
 }
 
 /* Row i of the softmax: fills p[0..i] (p[j] = 0 where not visible), returns lse. */
 static double softmax_row(const double* q, const double* k, long T, long D,
-                          double scale, long window, long i, double* p) {
+                          double scale, long window, long first, long i, double* p) {
     (void)T;
     double m = -INFINITY;
     for (long j = 0; j <= i; ++j) {
-        if (!visible(i, j, window)) { p[j] = -INFINITY; continue; }
+        if (!visible(i, j, window, first)) { p[j] = -INFINITY; continue; }
         double s = 0.0;
         for (long d = 0; d < D; ++d) s += q[i * D + d] * k[j * D + d];
         s *= scale;
@@ -67,18 +76,19 @@ static double softmax_row(const double* q, const double* k, long T, long D,
     }
     double sum = 0.0;
     for (long j = 0; j <= i; ++j)
-        if (visible(i, j, window)) sum += exp(p[j] - m);
+        if (visible(i, j, window, first)) sum += exp(p[j] - m);
     double lse = m + log(sum);
     for (long j = 0; j <= i; ++j)
-        p[j] = visible(i, j, window) ? exp(p[j] - lse) : 0.0;
+        p[j] = visible(i, j, window, first) ? exp(p[j] - lse) : 0.0;
     return lse;
 }
 
+/* first: per query row, the start of its document (NULL: one document). */
 static void fwd_head(const double* q, const double* k, const double* v,
-                     long T, long D, double scale, long window,
+                     long T, long D, double scale, long window, const long* first,
                      double* o, double* lse, double* p) {
     for (long i = 0; i < T; ++i) {
-        lse[i] = softmax_row(q, k, T, D, scale, window, i, p);
+        lse[i] = softmax_row(q, k, T, D, scale, window, first ? first[i] : 0, i, p);
         for (long d = 0; d < D; ++d) {
             double acc = 0.0;
             for (long j = 0; j <= i; ++j) acc += p[j] * v[j * D + d];
@@ -89,18 +99,19 @@ static void fwd_head(const double* q, const double* k, const double* v,
 
 static void bwd_head(const double* q, const double* k, const double* v,
                      const double* dO, long T, long D, double scale, long window,
-                     double* dq, double* dk, double* dv, double* delta,
-                     double* p, double* dp) {
+                     const long* first, double* dq, double* dk, double* dv,
+                     double* delta, double* p, double* dp) {
     memset(dk, 0, sizeof(double) * T * D);
     memset(dv, 0, sizeof(double) * T * D);
     for (long i = 0; i < T; ++i) {
-        softmax_row(q, k, T, D, scale, window, i, p);
+        const long fi = first ? first[i] : 0;
+        softmax_row(q, k, T, D, scale, window, fi, i, p);
         /* dV_j += P_ij dO_i ; dP_ij = dO_i . V_j */
         for (long j = 0; j <= i; ++j) {
             if (p[j] != 0.0)
                 for (long d = 0; d < D; ++d) dv[j * D + d] += p[j] * dO[i * D + d];
             double s = 0.0;
-            if (visible(i, j, window))
+            if (visible(i, j, window, fi))
                 for (long d = 0; d < D; ++d) s += dO[i * D + d] * v[j * D + d];
             dp[j] = s;
         }
@@ -123,11 +134,24 @@ static int bad_args(long NH, long T, long D) {
     return NH < 0 || T < 0 || D <= 0;
 }
 
-/* Returns 0 on success, 1 on bad arguments, 2 on allocation failure. */
-int oracle_attn_fwd(const double* q, const double* k, const double* v,
-                    long NH, long T, long D, double scale, long window,
-                    double* o, double* lse, int nthreads) {
-    if (bad_args(NH, T, D)) return 1;
+/* A document-start row must name, for every token, a position at or before it. */
+static int bad_doc_start(const long* doc_start, long NB, long T) {
+    if (!doc_start) return 0;
+    for (long n = 0; n < NB * T; ++n)
+        if (doc_start[n] < 0 || doc_start[n] > n % T) return 1;
+    return 0;
+}
+
+/* Heads are numbered h = b * H + hh (b batch row, hh head within the row).
+ * head_window: H windows, one per head position hh, or NULL for `window`
+ * everywhere.  doc_start: [NB, T] document starts, or NULL for one document
+ * per row.  Returns 0 on success, 1 on bad arguments, 2 on allocation failure. */
+int oracle_attn_fwd_masked(const double* q, const double* k, const double* v,
+                           long NB, long H, long T, long D, double scale,
+                           const long* head_window, long window, const long* doc_start,
+                           double* o, double* lse, int nthreads) {
+    if (NB < 0 || H <= 0 || bad_args(NB * H, T, D) || bad_doc_start(doc_start, NB, T)) return 1;
+    const long NH = NB * H;
     if (NH == 0 || T == 0) return 0;
     int fail = 0;
 #ifdef _OPENMP
@@ -142,8 +166,10 @@ int oracle_attn_fwd(const double* q, const double* k, const double* v,
 #endif
         for (long h = 0; h < NH; ++h) {
             if (!p) continue;
+            const long w = head_window ? head_window[h % H] : window;
+            const long* first = doc_start ? doc_start + (h / H) * T : NULL;
             fwd_head(q + h * T * D, k + h * T * D, v + h * T * D, T, D, scale,
-                     window, o + h * T * D, lse + h * T, p);
+                     w, first, o + h * T * D, lse + h * T, p);
         }
         free(p);
     }
@@ -151,11 +177,12 @@ int oracle_attn_fwd(const double* q, const double* k, const double* v,
     return fail ? 2 : 0;
 }
 
-int oracle_attn_bwd(const double* q, const double* k, const double* v,
-                    const double* dO, long NH, long T, long D, double scale,
-                    long window, double* dq, double* dk, double* dv,
-                    double* delta, int nthreads) {
-    if (bad_args(NH, T, D)) return 1;
+int oracle_attn_bwd_masked(const double* q, const double* k, const double* v,
+                           const double* dO, long NB, long H, long T, long D, double scale,
+                           const long* head_window, long window, const long* doc_start,
+                           double* dq, double* dk, double* dv, double* delta, int nthreads) {
+    if (NB < 0 || H <= 0 || bad_args(NB * H, T, D) || bad_doc_start(doc_start, NB, T)) return 1;
+    const long NH = NB * H;
     if (NH == 0 || T == 0) return 0;
     int fail = 0;
 #ifdef _OPENMP
@@ -171,8 +198,10 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v,
 #endif
         for (long h = 0; h < NH; ++h) {
             if (!p || !dp) continue;
+            const long w = head_window ? head_window[h % H] : window;
+            const long* first = doc_start ? doc_start + (h / H) * T : NULL;
             bwd_head(q + h * T * D, k + h * T * D, v + h * T * D, dO + h * T * D,
-                     T, D, scale, window, dq + h * T * D, dk + h * T * D,
+                     T, D, scale, w, first, dq + h * T * D, dk + h * T * D,
                      dv + h * T * D, delta + h * T, p, dp);
         }
         free(p);
@@ -180,6 +209,23 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v,
     }
     (void)nthreads;
     return fail ? 2 : 0;
+}
+
+/* Every head with the one window and no document boundaries. */
+int oracle_attn_fwd(const double* q, const double* k, const double* v,
+                    long NH, long T, long D, double scale, long window,
+                    double* o, double* lse, int nthreads) {
+    if (bad_args(NH, T, D)) return 1;
+    return oracle_attn_fwd_masked(q, k, v, NH, 1, T, D, scale, NULL, window, NULL, o, lse, nthreads);
+}
+
+int oracle_attn_bwd(const double* q, const double* k, const double* v,
+                    const double* dO, long NH, long T, long D, double scale,
+                    long window, double* dq, double* dk, double* dv,
+                    double* delta, int nthreads) {
+    if (bad_args(NH, T, D)) return 1;
+    return oracle_attn_bwd_masked(q, k, v, dO, NH, 1, T, D, scale, NULL, window, NULL, dq, dk, dv,
+                                  delta, nthreads);
 }
 
 int oracle_max_threads(void) {

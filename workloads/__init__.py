@@ -139,3 +139,37 @@ def sample_heads(B, H, n, seed=0):
 
 def default_scale(D: int) -> float:
     return 1.0 / math.sqrt(D)
+
+
+def doc_starts_from_lengths(lengths, T):
+    """[T] int32: for each position, the first position of the document holding it, for documents
+    of the given lengths laid end to end (the last one is cut at T)."""
+    import numpy as np
+    out = np.zeros(T, dtype=np.int32)
+    pos = 0
+    for n in lengths:
+        if pos >= T:
+            break
+        n = int(n)
+        if n < 1:
+            raise ValueError("document lengths must be >= 1")
+        out[pos:pos + n] = pos
+        pos += n
+    if pos < T:
+        out[pos:] = pos
+    return out
+
+
+def make_doc_starts(B, T, seed, max_doc_len, min_doc_len=1):
+    """[B, T] int32 document starts for B rows of T tokens packed with documents whose lengths are
+    drawn uniformly from [min_doc_len, max_doc_len] (one CPU torch.Generator seeded with `seed`).
+    Stands in for training batches aligned to end-of-document tokens with a maximum document
+    length (the modded-nanogpt README's technique list); no text is involved."""
+    import numpy as np
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    rows = []
+    for _ in range(B):
+        n = torch.randint(min_doc_len, max_doc_len + 1, (T,), generator=g).tolist()
+        rows.append(doc_starts_from_lengths(n, T))
+    return np.stack(rows).astype(np.int32)
