@@ -34,7 +34,7 @@ GPT_ATTN_ERR_WORKSPACE = 7
 
 EXPORTED = ("gpt_attn_fwd", "gpt_attn_bwd", "gpt_attn_bwd_workspace_bytes", "gpt_attn_bwd_delta",
             "gpt_attn_bwd_grads", "gpt_attn_bwd_dq_convert", "gpt_attn_check", "gpt_attn_status_string",
-            "gpt_attn_debug_wait_timeout", "gpt_attn_bwd_noalloc")
+            "gpt_attn_debug_wait_timeout", "gpt_attn_bwd_noalloc", "gpt_attn_tmap_cache_stats")
 
 _lib = None
 
@@ -72,6 +72,9 @@ def lib() -> ctypes.CDLL:
         L.gpt_attn_status_string.restype = ctypes.c_char_p
         L.gpt_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
         L.gpt_attn_bwd_noalloc.restype = i
+        L.gpt_attn_tmap_cache_stats.argtypes = [ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_longlong),
+                                                 ctypes.POINTER(ctypes.c_int)]
+        L.gpt_attn_tmap_cache_stats.restype = None
         L.gpt_attn_debug_wait_timeout.argtypes = [i, vp]
         L.gpt_attn_debug_wait_timeout.restype = i
         _lib = L
@@ -220,6 +223,13 @@ def gpt_attn_bwd_dq_convert(dq, workspace, scale=None, stream=None):
 def gpt_attn_check(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return int(lib().gpt_attn_check(_stream_handle(stream)))
+
+
+def gpt_attn_tmap_cache_stats():
+    """(hits, misses, entries) of the library's host-side tensor-map cache."""
+    h, m, u = ctypes.c_longlong(0), ctypes.c_longlong(0), ctypes.c_int(0)
+    lib().gpt_attn_tmap_cache_stats(ctypes.byref(h), ctypes.byref(m), ctypes.byref(u))
+    return h.value, m.value, u.value
 
 
 def gpt_attn_debug_wait_timeout(timeout_us: int, stream=None) -> int:

@@ -6,12 +6,14 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "attn_bwd.cuh"
 #include "attn_bwd_d64.cuh"
 #include "attn_fwd.cuh"
 #include "gpt_attn.h"
+#include "tmap_cache.h"
 
 extern "C" size_t gpt_attn_bwd_workspace_bytes(int B, int H, int T, int D);
 
@@ -49,35 +51,43 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// bf16 [BH, T, D] viewed as a 3-D tensor (D, T, BH); 64-column x 128-row boxes,
-// 128-byte swizzle (matches the UMMA 128B-swizzle canonical layout), zero fill
-// outside the tensor so ragged tails read as zeros.
-bool make_tmap_bf16(CUtensorMap* m, const void* base, int BH, int T, int D) {
+// Encodes the tensor map of `key` (see TmapKind): a 3-D view (D, T, BH) of a
+// row-major [BH, T, D] tensor, 128-row boxes whose width is 128 bytes of
+// elements (64 bf16 or 32 fp32 columns), 128-byte swizzle (the UMMA canonical
+// 128B-swizzled layout), zero fill outside the tensor so ragged tails read as zeros.
+bool encode_tmap(const TmapKey& key, CUtensorMap* m) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    const bool f32 = key.kind == (int)TmapKind::kF32Box32x128;
+    const cuuint64_t esz = f32 ? 4 : 2;
+    cuuint64_t dims[3] = {(cuuint64_t)key.d0, (cuuint64_t)key.d1, (cuuint64_t)key.d2};
+    cuuint64_t strides[2] = {(cuuint64_t)key.d0 * esz, (cuuint64_t)key.d1 * key.d0 * esz};
+    cuuint32_t box[3] = {f32 ? 32u : 64u, 128, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    reinterpret_cast<void*>(key.base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-// fp32 dQ accumulator [BH, T, D] as a 3-D tensor (D, T, BH); 32-column x 128-row boxes
-// (128 bytes wide, 128-byte swizzle) for the bulk reduce-add.
+TmapCache<CUtensorMap>& tmap_cache() {
+    static TmapCache<CUtensorMap> c;
+    return c;
+}
+
+bool cached_tmap(CUtensorMap* m, const void* base, TmapKind kind, int BH, int T, int D) {
+    const TmapKey key{reinterpret_cast<uintptr_t>(base), (int)kind, D, T, BH};
+    return tmap_cache().get(key, m, [](const TmapKey& k, CUtensorMap* v) { return encode_tmap(k, v); });
+}
+
+// bf16 [BH, T, D]; 64-column x 128-row boxes.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, int BH, int T, int D) {
+    return cached_tmap(m, base, TmapKind::kBf16Box64x128, BH, T, D);
+}
+
+// fp32 dQ accumulator [BH, T, D]; 32-column x 128-row boxes for the bulk reduce-add.
 bool make_tmap_f32_acc(CUtensorMap* m, const void* base, int BH, int T, int D) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)T * D * 4};
-    cuuint32_t box[3] = {32, 128, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return cached_tmap(m, base, TmapKind::kF32Box32x128, BH, T, D);
 }
 
 bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
@@ -153,16 +163,18 @@ WsLayout ws_layout(void* ws, int BH, int T, int D) {
     return w;
 }
 
+// SM count of the current device, cached per device.  Host threads may call the library at the
+// same time: the cache entries are atomics (every thread would store the same value).
 int sm_count() {
-    static int counts[64] = {};
+    static std::atomic<int> counts[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (counts[dev] == 0) {
-        int n = 0;
+    int n = counts[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        counts[dev] = n;
+        counts[dev].store(n, std::memory_order_relaxed);
     }
-    return counts[dev];
+    return n;
 }
 
 int launch_bwd_delta(const void* o, const float* lse, const void* dout, int BH, int T, int D, void* ws,
@@ -260,28 +272,20 @@ __global__ void debug_wait_kernel(uint64_t timeout_ns) {
 // created when the library's module is loaded on a device and lives until the
 // process exits, so the entry point below never allocates.  In host code the
 // name g_noalloc_scratch is only a host-side shadow symbol, not a device
-// address: the device address is looked up with cudaGetSymbolAddress, once
-// per device, with that device current.
+// address: the device address is looked up with cudaGetSymbolAddress with the
+// caller's device current.
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (looked up on the
-// first call per device), or nullptr on a CUDA error.
+// Device address of the scratch array on the current device, or nullptr on a
+// CUDA error.  Looked up on every call (a table lookup once the module is
+// loaded) rather than cached: after a cudaDeviceReset the module is loaded
+// again and the array may live at a different address.
 void* noalloc_scratch_current_device() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
-        g_scratch_addr[dev] = ptr;
-    }
-    return g_scratch_addr[dev];
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    return ptr;
 }
 }  // namespace
 }  // namespace gpt_attn
@@ -400,6 +404,15 @@ int gpt_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void
     // rewrite every byte they read (dQ accumulator zeroed, row vectors written
     // including padding), so nothing else needs clearing here.
     return gpt_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, window, ws, need, stream);
+}
+
+void gpt_attn_tmap_cache_stats(long long* hits, long long* misses, int* entries) {
+    long long h = 0, m = 0;
+    int u = 0;
+    gpt_attn::tmap_cache().stats(&h, &m, &u);
+    if (hits) *hits = h;
+    if (misses) *misses = m;
+    if (entries) *entries = u;
 }
 
 int gpt_attn_debug_wait_timeout(int timeout_us, void* stream) {

@@ -157,6 +157,16 @@ int gpt_attn_check(void* stream);
 const char* gpt_attn_status_string(int status);
 
 /*
+ * Counters of the host-side tensor-map cache.  Every call encodes the TMA
+ * descriptors of its tensors from (base address, element type, B*H, T, D);
+ * an encoded descriptor depends on nothing else, so the library keeps the
+ * last 64 in host memory and repeated calls on the same buffers skip the
+ * encoding.  Reports the lookups served from the cache, the encodings done,
+ * and the entries held (any pointer may be NULL).  Host only, thread-safe.
+ */
+void gpt_attn_tmap_cache_stats(long long* hits, long long* misses, int* entries);
+
+/*
  * Diagnostic: launches one small kernel that waits on a shared-memory
  * barrier nothing ever arrives at, with a bound of `timeout_us` microseconds.
  * The wait runs out, the kernel records GPT_ATTN_ERR_TIMEOUT in the status
