@@ -59,6 +59,8 @@ def _load():
         lib.oracle_attn_bwd_masked.argtypes = [dp, dp, dp, dp, L, L, L, L, ctypes.c_double, lp, L, lp,
                                                dp, dp, dp, dp, ctypes.c_int]
         lib.oracle_attn_bwd_masked.restype = ctypes.c_int
+        lib.oracle_attn_decode.argtypes = [dp, dp, dp, lp, L, L, L, L, ctypes.c_double, L, dp, dp, ctypes.c_int]
+        lib.oracle_attn_decode.restype = ctypes.c_int
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -163,3 +165,20 @@ def attn_bwd_masked(q, k, v, dO, scale: float, head_windows=None, window: int = 
     if rc != 0:
         raise RuntimeError(f"oracle_attn_bwd_masked failed with code {rc}")
     return dq, dk, dv, delta
+
+
+def attn_decode(q, k_cache, v_cache, lens, scale: float, window: int = 0, nthreads: int = 0):
+    """Decode: q [B, H, D] against cached keys/values [B, H, T_max, D]; sequence b has lens[b]
+    tokens and its query is the last one.  Returns (O [B, H, D], lse [B, H]) in fp64."""
+    q, k, v = _as_f64(q), _as_f64(k_cache), _as_f64(v_cache)
+    if q.ndim != 3 or k.ndim != 4 or k.shape != v.shape or k.shape[:2] != q.shape[:2] or k.shape[3] != q.shape[2]:
+        raise ValueError("q must be [B, H, D] and the caches [B, H, T_max, D]")
+    B, H, T, D = k.shape
+    ln, lnp = _long_array(lens, B)
+    o = np.zeros_like(q)
+    lse = np.zeros((B, H), dtype=np.float64)
+    rc = _load().oracle_attn_decode(_ptr(q), _ptr(k), _ptr(v), lnp, B, H, T, D, float(scale), int(window),
+                                    _ptr(o), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_decode failed with code {rc}")
+    return o, lse

@@ -228,6 +228,59 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v,
                                   delta, nthreads);
 }
 
+/* Decode: one new query per (b, h) against its cached keys and values, as the
+ * generation loop of "Un GPT desde cero + nanoGPT" (Laboratorio L2.1, generate)
+ * runs the model on the growing sequence and keeps only the last position.  The
+ * query is the last token of a sequence of length L = lens[b] (clamped to
+ * [0, T_max]); it sees keys j < L, and with a window W >= 1 only j >= L - W.
+ *   q: [NB*H, D]; k, v: [NB*H, T_max, D]; o: [NB*H, D]; lse: [NB*H] (natural log;
+ *   -inf and o = 0 when no key is visible).
+ * Returns 0 on success, 1 on bad arguments. */
+int oracle_attn_decode(const double* q, const double* k, const double* v, const long* lens,
+                       long NB, long H, long T_max, long D, double scale, long window,
+                       double* o, double* lse, int nthreads) {
+    if (NB < 0 || H <= 0 || T_max < 0 || D <= 0 || !lens) return 1;
+    const long NH = NB * H;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+#endif
+    for (long h = 0; h < NH; ++h) {
+        long L = lens[h / H];
+        if (L < 0) L = 0;
+        if (L > T_max) L = T_max;
+        const long lo = (window > 0 && L - window > 0) ? L - window : 0;
+        const double* qh = q + h * D;
+        const double* kh = k + h * T_max * D;
+        const double* vh = v + h * T_max * D;
+        double m = -INFINITY;
+        for (long j = lo; j < L; ++j) {
+            double s = 0.0;
+            for (long d = 0; d < D; ++d) s += qh[d] * kh[j * D + d];
+            s *= scale;
+            if (s > m) m = s;
+        }
+        for (long d = 0; d < D; ++d) o[h * D + d] = 0.0;
+        if (L <= lo) { lse[h] = -INFINITY; continue; }
+        double sum = 0.0;
+        for (long j = lo; j < L; ++j) {
+            double s = 0.0;
+            for (long d = 0; d < D; ++d) s += qh[d] * kh[j * D + d];
+            sum += exp(s * scale - m);
+        }
+        const double l = m + log(sum);
+        lse[h] = l;
+        for (long j = lo; j < L; ++j) {
+            double s = 0.0;
+            for (long d = 0; d < D; ++d) s += qh[d] * kh[j * D + d];
+            const double p = exp(s * scale - l);
+            for (long d = 0; d < D; ++d) o[h * D + d] += p * vh[j * D + d];
+        }
+    }
+    (void)nthreads;
+    return 0;
+}
+
 int oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
