@@ -46,6 +46,9 @@ def parse_args():
                     help="workload number (1-5); the default is the headline shape")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--decode", action="store_true",
+                    help="time decode attention instead (one new query per sequence against a K/V cache; "
+                         "GB/s of cache read against the HBM peak) and print its own JSON line")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 256 MB buffer between timed steps (outside their events) and sum the "
                          "per-step times: a cold-L2 figure for workloads whose inputs fit in L2")
@@ -280,8 +283,51 @@ def workload_config(w):
                            else "algorithmic: 4*D per visible pair fwd, 10*D bwd")}
 
 
+def run_decode(args):
+    """Decode attention for generation: B sequences of a GPT-2 124M-shaped K/V cache (H=12, D=64,
+    T_max=1024), each at full length, one new query each.  Memory-bound: reports the K/V bytes read
+    per call over the call's device time against the HBM peak."""
+    import torch
+    import causal_attention_sdpa_b200 as ga
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    lines = []
+    for B, H, T, D in ((64, 12, 1024, 64), (1, 12, 1024, 64), (16, 6, 8192, 128)):
+        q4, k, v, _ = workloads.make_inputs(B, H, T, D, seed=77, device=dev)
+        q = q4[:, :, -1].contiguous()
+        lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(16, ga.gpt_attn_decode_workspace_bytes(B, H, T, D)), dtype=torch.uint8, device=dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for _ in range(args.warmup):
+            ga.gpt_attn_decode(q, k, v, lens, o=o, lse=lse, workspace=ws)
+        assert ga.gpt_attn_check() == ga.GPT_ATTN_OK
+        times = []
+        for _ in range(args.steps):
+            flush.zero_()                        # cold L2: the caches come from HBM, as in generation
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            ga.gpt_attn_decode(q, k, v, lens, o=o, lse=lse, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        nbytes = 2 * B * H * T * D * 2 + 2 * B * H * D * 2 + B * H * 4
+        lines.append({"B": B, "H": H, "T_max": T, "D": D, "ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9,
+                      "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]})
+    print(json.dumps({"metric": "decode attention K/V-cache read bandwidth on 1 B200", "unit": "GB/s",
+                      "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                      "l2": "256 MB written between calls (outside the events)", "steps": args.steps,
+                      "warmup": args.warmup, "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"],
+                      "cases": lines}), flush=True)
+
+
 def main():
     args = parse_args()
+    if args.decode:
+        return run_decode(args)
     w = workloads.BY_INDEX[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -362,6 +408,7 @@ def main():
     per_kernel = {name: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps
                   for i, name in enumerate(("attn_fwd_kernel", "attn_bwd_prep_kernel", "attn_bwd_kernel",
                                             "attn_dq_convert_kernel"))}
+    step_median_ms = max_over_ranks(statistics.median(e[0].elapsed_time(e[4]) for e in evs), dist, dev)
     total_ms = max_over_ranks(total_ms, dist, dev)
 
     flops_step = workloads.fwd_bwd_flops(B, H, T, D, w.window)
@@ -437,6 +484,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "ms_per_step_median": step_median_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": dict(workload_config(w), **({"l2": "L2 flushed between steps (256 MB "
                                                                     "write outside the step events), "

@@ -31,10 +31,21 @@ GPT_ATTN_ERR_ALIGN = 4
 GPT_ATTN_ERR_CUDA = 5
 GPT_ATTN_ERR_TIMEOUT = 6
 GPT_ATTN_ERR_WORKSPACE = 7
+GPT_ATTN_ERR_UNAVAILABLE = 8
+GPT_ATTN_ERR_BOUNDS = 9
 
 EXPORTED = ("gpt_attn_fwd", "gpt_attn_bwd", "gpt_attn_bwd_workspace_bytes", "gpt_attn_bwd_delta",
             "gpt_attn_bwd_grads", "gpt_attn_bwd_dq_convert", "gpt_attn_check", "gpt_attn_status_string",
-            "gpt_attn_debug_wait_timeout", "gpt_attn_bwd_noalloc", "gpt_attn_tmap_cache_stats")
+            "gpt_attn_debug_wait_timeout", "gpt_attn_bwd_noalloc", "gpt_attn_tmap_cache_stats",
+            "gpt_attn_fwd_masked", "gpt_attn_bwd_masked", "gpt_attn_decode", "gpt_attn_decode_workspace_bytes",
+            "gpt_attn_debug_skip_load")
+
+
+class GptAttnMask(ctypes.Structure):
+    """The C ABI's gpt_attn_mask: a window for every head, or per-head windows (host ints), and
+    optional document starts (device int32 [B, T])."""
+    _fields_ = [("window", ctypes.c_int), ("head_windows", ctypes.POINTER(ctypes.c_int)),
+                ("doc_start", ctypes.c_void_p)]
 
 _lib = None
 
@@ -75,6 +86,17 @@ def lib() -> ctypes.CDLL:
         L.gpt_attn_tmap_cache_stats.argtypes = [ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_longlong),
                                                  ctypes.POINTER(ctypes.c_int)]
         L.gpt_attn_tmap_cache_stats.restype = None
+        mp = ctypes.POINTER(GptAttnMask)
+        L.gpt_attn_fwd_masked.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, mp, vp]
+        L.gpt_attn_fwd_masked.restype = i
+        L.gpt_attn_bwd_masked.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, mp, vp, sz, vp]
+        L.gpt_attn_bwd_masked.restype = i
+        L.gpt_attn_decode_workspace_bytes.argtypes = [i, i, i, i, i]
+        L.gpt_attn_decode_workspace_bytes.restype = sz
+        L.gpt_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+        L.gpt_attn_decode.restype = i
+        L.gpt_attn_debug_skip_load.argtypes = [i]
+        L.gpt_attn_debug_skip_load.restype = i
         L.gpt_attn_debug_wait_timeout.argtypes = [i, vp]
         L.gpt_attn_debug_wait_timeout.restype = i
         _lib = L
@@ -176,6 +198,67 @@ def gpt_attn_bwd_noalloc(q, k, v, o, lse, dO, scale=None, window=0, dq=None, dk=
     return dq, dk, dv
 
 
+def _mask(H, window=0, head_windows=None, doc_start=None):
+    """A GptAttnMask (and the host array it points at, which must outlive the call)."""
+    import torch
+    hw = None
+    if head_windows is not None:
+        hw = (ctypes.c_int * H)(*[int(x) for x in head_windows])
+        if len(head_windows) != H:
+            raise ValueError(f"head_windows needs {H} entries")
+    if doc_start is not None:
+        if doc_start.dtype != torch.int32 or not doc_start.is_cuda or not doc_start.is_contiguous():
+            raise ValueError("doc_start must be a contiguous CUDA int32 tensor [B, T]")
+    m = GptAttnMask(int(window), ctypes.cast(hw, ctypes.POINTER(ctypes.c_int)) if hw is not None else None,
+                    doc_start.data_ptr() if doc_start is not None else None)
+    return m, hw
+
+
+def gpt_attn_fwd_masked(q, k, v, scale=None, window=0, head_windows=None, doc_start=None, o=None, lse=None,
+                        stream=None):
+    """Forward pass with per-head windows and/or document starts; returns (o, lse)."""
+    import torch
+    B, H, T, D = q.shape
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_bf16(n, t, q.shape)
+    if doc_start is not None and tuple(doc_start.shape) != (B, T):
+        raise ValueError(f"doc_start must have shape {(B, T)}")
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
+    m, keep = _mask(H, window, head_windows, doc_start)
+    rc = lib().gpt_attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, D, float(scale),
+                                   ctypes.byref(m), _stream_handle(stream))
+    del keep
+    if rc != GPT_ATTN_OK:
+        raise GptAttnError(rc, "gpt_attn_fwd_masked")
+    return o, lse
+
+
+def gpt_attn_bwd_masked(q, k, v, o, lse, dO, scale=None, window=0, head_windows=None, doc_start=None, dq=None,
+                        dk=None, dv=None, workspace=None, stream=None):
+    """Backward pass under the same mask as gpt_attn_fwd_masked; returns (dq, dk, dv)."""
+    import torch
+    B, H, T, D = q.shape
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO)):
+        _check_bf16(n, t, q.shape)
+    if doc_start is not None and tuple(doc_start.shape) != (B, T):
+        raise ValueError(f"doc_start must have shape {(B, T)}")
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    ws, nbytes = _ws(workspace, q)
+    m, keep = _mask(H, window, head_windows, doc_start)
+    rc = lib().gpt_attn_bwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), B, H, T, D, float(scale), ctypes.byref(m), _ptr(ws), nbytes,
+                                   _stream_handle(stream))
+    del keep
+    if rc != GPT_ATTN_OK:
+        raise GptAttnError(rc, "gpt_attn_bwd_masked")
+    return dq, dk, dv
+
+
 def _ws(workspace, q):
     import torch
     B, H, T, D = q.shape
@@ -218,6 +301,35 @@ def gpt_attn_bwd_dq_convert(dq, workspace, scale=None, stream=None):
                                        _stream_handle(stream))
     if rc != GPT_ATTN_OK:
         raise GptAttnError(rc, "gpt_attn_bwd_dq_convert")
+
+
+def gpt_attn_decode_workspace_bytes(B, H, T_max, D, window=0) -> int:
+    return int(lib().gpt_attn_decode_workspace_bytes(int(B), int(H), int(T_max), int(D), int(window)))
+
+
+def gpt_attn_decode(q, k_cache, v_cache, seq_lens, scale=None, window=0, o=None, lse=None, workspace=None,
+                    stream=None):
+    """Decode: q bf16 [B, H, D] against caches bf16 [B, H, T_max, D]; seq_lens int32 [B] on the
+    device.  Returns (o [B, H, D], lse [B, H])."""
+    import torch
+    B, H, T, D = k_cache.shape
+    _check_bf16("k_cache", k_cache, (B, H, T, D))
+    _check_bf16("v_cache", v_cache, (B, H, T, D))
+    _check_bf16("q", q, (B, H, D))
+    if seq_lens.dtype != torch.int32 or not seq_lens.is_cuda or tuple(seq_lens.shape) != (B,):
+        raise ValueError("seq_lens must be a CUDA int32 tensor [B]")
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = gpt_attn_decode_workspace_bytes(B, H, T, D, window)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    rc = lib().gpt_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), _ptr(o), _ptr(lse), B, H,
+                               T, D, float(scale), int(window), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if rc != GPT_ATTN_OK:
+        raise GptAttnError(rc, "gpt_attn_decode")
+    return o, lse
 
 
 def gpt_attn_check(stream=None) -> int:

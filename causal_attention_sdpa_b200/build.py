@@ -13,6 +13,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgpt_attn.so")
+DEBUG_LIB = os.path.join(PKG, "libgpt_attn_debug.so")   # -DGPT_ATTN_DEBUG: bounds checks, load-skip hook
 SOURCES = [os.path.join(CSRC, "gpt_attn.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + \
     [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
@@ -25,29 +26,33 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def command(out: str, verbose: bool = False):
+def command(out: str, verbose: bool = False, debug: bool = False):
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
            "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC, "-o", out] + SOURCES
+    if debug:
+        cmd.insert(1, "-DGPT_ATTN_DEBUG")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     return cmd
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if force or not up_to_date():
-        tmp = LIB + f".tmp{os.getpid()}"
-        subprocess.run(command(tmp, verbose), check=True)
-        os.replace(tmp, LIB)
-    return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Build the library (or, with debug=True, libgpt_attn_debug.so) if a source is newer."""
+    lib = DEBUG_LIB if debug else LIB
+    if force or not up_to_date(lib):
+        tmp = lib + f".tmp{os.getpid()}"
+        subprocess.run(command(tmp, verbose, debug), check=True)
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
-    print(LIB)
+    debug = "--debug" in sys.argv
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, debug=debug))

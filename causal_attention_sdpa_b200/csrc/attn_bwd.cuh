@@ -46,15 +46,22 @@ struct BwdParams {
     int* sched;             // work-unit counter of the persistent kernel, zeroed by the prep kernel
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
+    // Document masks only (else nullptr), written by the prep kernel into the workspace:
+    const int* lower2;      // [BH, T_pad]   lower bound of each row's visible keys; INT_MAX past T
+    const int* last_qt;     // [BH, n_tiles] last query tile that sees each key tile
     int T;
     int T_pad;
     int BH;
     int n_tiles;
-    int window;
     float scale_log2;       // scale * log2(e)
     float scale;
     uint64_t timeout_ns;
 };
+
+// Last query tile that sees key tile kt of head bh (window W).
+__device__ __forceinline__ int bwd_last_tile(const BwdParams& p, int bh, int kt, int W) {
+    return p.last_qt ? __ldg(p.last_qt + (size_t)bh * p.n_tiles + kt) : bwd_last_query_tile(kt, p.n_tiles, W);
+}
 
 template <int D>
 struct BwdCfg {
@@ -78,6 +85,7 @@ struct BwdSmem {
     alignas(1024) uint8_t ds[kTile * kTile * 2];           // dS^T bf16 [key][query], two 64-query halves
     alignas(16) float lse2[C::kStages][kTile];
     alignas(16) float delta[C::kStages][kTile];
+    alignas(16) int lower[C::kStages][kTile];               // document masks only
     uint64_t bar_kv;
     uint64_t bar_qdo_full[C::kStages];
     uint64_t bar_qdo_empty[C::kStages];
@@ -98,12 +106,18 @@ struct BwdSmem {
 // Delta_i = dO_i . O_i, lse2_i = lse_i * log2(e) for every padded row, and a
 // zeroed fp32 dQ accumulator.  G = D / 8 threads per row, 16-byte accesses.
 // No thread leaves before the group shuffle (every lane of the warp takes part).
+// With document starts (lower2 != nullptr) it also writes each padded row's lower
+// bound of visible keys (INT_MAX past T) and, from the first row of each key tile,
+// the last query tile that sees the tile: the first rows' lower bounds do not
+// decrease, so the query tiles that see a key tile are the ones up to the last
+// whose first row's lower bound is at or before the tile's last key.
 template <int D>
 __global__ void __launch_bounds__(256)
 attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                      const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ delta,
                      float* __restrict__ dq_acc, int* __restrict__ sched, int T, int T_pad,
-                     long long total_rows_pad) {
+                     long long total_rows_pad, const MaskParams mask, int* __restrict__ lower2,
+                     int* __restrict__ last_qt, int n_tiles) {
     constexpr int G = D / 8;
     if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0;
     const long long row = (long long)blockIdx.x * (256 / G) + threadIdx.x / G;
@@ -135,6 +149,15 @@ attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* _
     if (in_range && g == 0) {
         delta[row] = valid ? acc : 0.f;
         lse2[row] = valid ? lse[bh * T + t] * 1.4426950408889634f : INFINITY;
+        if (lower2) {
+            const int W = mask_window(mask, (int)bh);
+            lower2[row] = valid ? mask_row_lower(mask, (int)bh, T, W, t) : INT_MAX;
+            if ((t & (kTile - 1)) == 0) {
+                const int b = (int)bh;
+                last_qt[bh * n_tiles + t / kTile] = bwd_last_query_tile_lb(
+                    t / kTile, n_tiles, [&](int qt) { return mask_row_lower(mask, b, T, W, qt * kTile); });
+            }
+        }
     }
 }
 
@@ -152,11 +175,11 @@ __global__ void attn_dq_convert_kernel(const float* __restrict__ acc, __nv_bfloa
     reinterpret_cast<uint4*>(dq)[i] = r;
 }
 
-template <int D>
+template <int D, typename Mask>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const BwdParams p) {
+                const BwdParams p, const __grid_constant__ Mask mask) {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(smem_align1024(smem_raw));
@@ -177,7 +200,8 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const int kt = blockIdx.x % p.n_tiles;
     const int k0 = kt * kTile;
     const int qt_lo = kt;
-    const int qt_hi = bwd_last_query_tile(kt, p.n_tiles, p.window);
+    const int W = mask.head_window(bh);
+    const int qt_hi = bwd_last_tile(p, bh, kt, W);
     const int n_q = qt_hi - qt_lo + 1;
 
     if (threadIdx.x == 0) {
@@ -228,7 +252,7 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const int n = it / kStages;
                 if (n > 0 && !mbar_wait(&sm.bar_qdo_empty[s], (n - 1) & 1, ac)) break;
                 const int q0 = (qt_lo + it) * kTile;
-                mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + 2 * kTile * 4);
+                mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + (p.lower2 ? 3 : 2) * kTile * 4);
                 for (int b = 0; b < kBoxes; ++b) {
                     tma_load_3d(sm.q[s] + b * 16384, &tm_q, &sm.bar_qdo_full[s], b * 64, q0, bh);
                     tma_load_3d(sm.dout[s] + b * 16384, &tm_do, &sm.bar_qdo_full[s], b * 64, q0, bh);
@@ -236,6 +260,7 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const size_t roff = (size_t)bh * p.T_pad + q0;
                 bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
                 bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_qdo_full[s]);
+                if (p.lower2) bulk_load(sm.lower[s], p.lower2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
             }
             if (sm.abort_flag) {
                 mbar_wait_drain(&sm.bar_kv, 0, p.timeout_ns);
@@ -319,8 +344,8 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         const int r = wq * 32 + lane;
         const int key = k0 + r;
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
-        const int W = p.window;
         const float sl2 = p.scale_log2;
+        const bool doc = p.lower2 != nullptr;
         const uint32_t ds_row = smem_u32(sm.ds) + r * 128;
         bool ok = true;
         for (int it = 0; it < n_q; ++it) {
@@ -333,7 +358,11 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             if (!warp_wait(&sm.bar_dp_full, it & 1, ac)) { ok = false; break; }
             if (it > 0 && !warp_wait(&sm.bar_ds_empty, (it - 1) & 1, ac)) { ok = false; break; }
             tc_fence_after();
-            const bool need_mask = (qt == kt) || (W > 0 && q0 + kTile - 1 >= k0 + W);
+            // The tile needs the per-element mask if it holds the diagonal or some query of it
+            // starts seeing keys after this key tile's first key (lower bounds do not decrease
+            // down a tile, so its last row decides).
+            const bool need_mask =
+                (qt == kt) || (doc ? sm.lower[s][kTile - 1] > k0 : (W > 0 && q0 + kTile - 1 >= k0 + W));
             const float2* lse2 = reinterpret_cast<const float2*>(sm.lse2[s]);
             const float2* dlt = reinterpret_cast<const float2*>(sm.delta[s]);
 #pragma unroll 1
@@ -343,13 +372,21 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 tmem_ld32(t_lane + C::kColDP + c * 32, rd);
                 tmem_wait_ld();
                 if (need_mask) {
-                    // visible query columns of this key: one range, compare + select per element
                     const int c_lo = key - (q0 + c * 32);
-                    const int c_hi = W > 0 ? key + W - 1 - (q0 + c * 32) : INT_MAX / 2;
-                    const uint32_t span = (uint32_t)(c_hi - c_lo);
+                    if (doc) {
+                        // query q sees this key iff q >= key and lower(q) <= key
+                        const int* lw = sm.lower[s] + c * 32;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        rs[e] = ((uint32_t)(e - c_lo) <= span) ? rs[e] : 0xff800000u;   // -inf: P = 0
+                        for (int e = 0; e < 32; ++e)
+                            rs[e] = (e >= c_lo && lw[e] <= key) ? rs[e] : 0xff800000u;   // -inf: P = 0
+                    } else {
+                        // visible query columns of this key: one range, compare + select per element
+                        const int c_hi = W > 0 ? key + W - 1 - (q0 + c * 32) : INT_MAX / 2;
+                        const uint32_t span = (uint32_t)(c_hi - c_lo);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            rs[e] = ((uint32_t)(e - c_lo) <= span) ? rs[e] : 0xff800000u;   // -inf: P = 0
+                    }
                 }
                 uint32_t pk[16], dk[16];
 #pragma unroll

@@ -61,6 +61,7 @@ struct Bwd64Smem {
     alignas(1024) uint8_t ds[2][kTile * kTile * 2];
     alignas(16) float lse2[C::kStages][kTile];
     alignas(16) float delta[C::kStages][kTile];
+    alignas(16) int lower[C::kStages][kTile];       // document masks only
     int unit[2];                  // work-unit ring: id, or -1 when there is no more work
     uint64_t bar_unit_full[2];
     uint64_t bar_unit_empty[2];
@@ -87,22 +88,28 @@ struct Bwd64Smem {
 };
 
 struct Bwd64Unit {
-    int bh, kt, k0, qt_lo, n_q;
+    int bh, kt, k0, qt_lo, n_q, W;
 };
 
-__device__ __forceinline__ Bwd64Unit bwd64_unit(int u, const BwdParams& p) {
+// Work unit u (head-major): head bh, key tile kt, and the n_q query tiles [kt, kt + n_q) that see it.
+template <typename Mask>
+__device__ __forceinline__ Bwd64Unit bwd64_unit(int u, const BwdParams& p, const Mask& mask) {
     Bwd64Unit w;
-    bwd_unit(u, p.n_tiles, p.window, w.bh, w.kt, w.n_q);   // schedule.h
+    w.bh = u / p.n_tiles;
+    w.kt = u % p.n_tiles;
+    w.W = mask.head_window(w.bh);
+    w.n_q = bwd_last_tile(p, w.bh, w.kt, w.W) - w.kt + 1;
     w.k0 = w.kt * kTile;
     w.qt_lo = w.kt;
     return w;
 }
 
+template <typename Mask>
 __global__ void __launch_bounds__(kBwd64Threads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk,
-                const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
+                const __grid_constant__ CUtensorMap tm_dv, const BwdParams p, const __grid_constant__ Mask mask) {
     using C = Bwd64Cfg;
     constexpr int D = C::D;
     extern __shared__ uint8_t smem_raw[];
@@ -189,7 +196,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 *reinterpret_cast<volatile int*>(&sm.unit[slot]) = u;
                 mbar_arrive(&sm.bar_unit_full[slot]);
                 if (u < 0) break;
-                const Bwd64Unit w = bwd64_unit(u, p);
+                const Bwd64Unit w = bwd64_unit(u, p, mask);
                 const int kb = n & 1;
                 if (n >= 2 && !(ok = mbar_wait(&sm.bar_kv_empty[kb], ((n >> 1) - 1) & 1, ac))) break;
                 mbar_arrive_expect_tx(&sm.bar_kv_full[kb], 2 * kTileBytes);
@@ -200,13 +207,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const int s = g % kStages;
                     const int m = g / kStages;
                     if (m > 0 && !(ok = mbar_wait(&sm.bar_qdo_empty[s], (m - 1) & 1, ac))) break;
+                    if (debug_skip_load(2, g)) continue;           // debug builds: exercise the abort path
                     const int q0 = (w.qt_lo + i) * kTile;
-                    mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + 2 * kTile * 4);
+                    mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + (p.lower2 ? 3 : 2) * kTile * 4);
                     tma_load_3d(sm.q[s], &tm_q, &sm.bar_qdo_full[s], 0, q0, w.bh);
                     tma_load_3d(sm.dout[s], &tm_do, &sm.bar_qdo_full[s], 0, q0, w.bh);
                     const size_t roff = (size_t)w.bh * p.T_pad + q0;
                     bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
                     bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_qdo_full[s]);
+                    if (p.lower2) bulk_load(sm.lower[s], p.lower2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
                 }
             }
             if (sm.abort_flag) {
@@ -223,7 +232,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int n = 0; ok; ++n) {
                 int u;
                 if (!(ok = read_unit(n, u)) || u < 0) break;
-                const Bwd64Unit w = bwd64_unit(u, p);
+                const Bwd64Unit w = bwd64_unit(u, p, mask);
                 const int kb = n & 1;
                 const uint32_t k_addr = smem_u32(sm.k[kb]);
                 const uint32_t v_addr = smem_u32(sm.v[kb]);
@@ -309,15 +318,16 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
-        const int W = p.window;
         const float sl2 = p.scale_log2;
+        const bool doc = p.lower2 != nullptr;
         bool ok = true;
         int g = 0;
         for (int n = 0; ok; ++n) {
             int u = -1;
             ok = __all_sync(0xffffffffu, read_unit(n, u));
             if (!ok || u < 0) break;
-            const Bwd64Unit w = bwd64_unit(u, p);
+            const Bwd64Unit w = bwd64_unit(u, p, mask);
+            const int W = w.W;
             const int key = w.k0 + r;
             for (int i = 0; i < w.n_q; ++i, ++g) {
                 const int s = g % kStages;
@@ -331,7 +341,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // The 64 query columns of this warpgroup are processed as two 32-column halves in a
                 // loop that is not unrolled (half the code of an unrolled pass); the second half's
                 // S^T and dP^T are read from TMEM while the first half is computed.
-                const bool need_mask = (qt == w.kt) || (W > 0 && qt * kTile + kTile - 1 >= w.k0 + W);
+                // The diagonal tile, and tiles some of whose queries start seeing keys after this
+                // key tile's first key (the tile's last row decides: lower bounds do not decrease).
+                const bool need_mask = (qt == w.kt) || (doc ? sm.lower[s][kTile - 1] > w.k0
+                                                            : (W > 0 && qt * kTile + kTile - 1 >= w.k0 + W));
                 // Query columns that see this key form one range [c_lo, c_hi] (query >= key, and
                 // query < key + W under a window): blocked pairs get score -inf, hence P = dS = 0.
                 const int c_lo = key - qc0;
@@ -345,9 +358,17 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     if (need_mask) {
+                        if (doc) {
+                            // query column c sees this key iff c >= c_lo and lower(c) <= key
+                            const int* lw = sm.lower[s] + h * 64 + hh * 32;
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            xs[e] = ((uint32_t)(hh * 32 + e - c_lo) <= span) ? xs[e] : 0xff800000u;   // -inf
+                            for (int e = 0; e < 32; ++e)
+                                xs[e] = (hh * 32 + e >= c_lo && lw[e] <= key) ? xs[e] : 0xff800000u;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                xs[e] = ((uint32_t)(hh * 32 + e - c_lo) <= span) ? xs[e] : 0xff800000u;   // -inf
+                        }
                     }
                     const float4* lse4 = reinterpret_cast<const float4*>(sm.lse2[s] + h * 64 + hh * 32);
                     const float4* dl4 = reinterpret_cast<const float4*>(sm.delta[s] + h * 64 + hh * 32);
@@ -416,7 +437,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             int u = -1;
             ok = __all_sync(0xffffffffu, read_unit(n, u));
             if (!ok || u < 0) break;
-            const Bwd64Unit w = bwd64_unit(u, p);
+            const Bwd64Unit w = bwd64_unit(u, p, mask);
             const int kb = n & 1;
             // dK / dV of this unit (thread = key row): copied out of TMEM as soon as the unit's last
             // dQ is complete, before that dQ is reduced, so the next unit's first dV/dK can start.
@@ -500,7 +521,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
         }
-        if (warp == 12 && lane == 0) bulk_wait_group0();   // every reduce has landed in global memory
+        if (warp == 12 && lane == 0) bulk_wait_group0();   // every reduce and store has landed
     }
 
     tc_fence_before();

@@ -48,6 +48,42 @@ namespace gpt_attn {
 constexpr int kFwdThreads = 384;
 constexpr float kLazyRescale = 8.0f; // log2 units
 
+// Which keys each query sees, shared by the forward and backward kernels.  The kernels are
+// instantiated for two mask types with the same interface: WindowMask (causal, or one window for
+// every head: the common case, with nothing but one integer in the kernel parameters) and
+// MaskParams (a window per head position h = bh % H, and optional document starts [B, T] in
+// device memory, row b = bh / H).
+struct WindowMask {
+    int window;                // <= 0: causal only
+    __device__ __forceinline__ int head_window(int) const { return window; }
+    // Lower bound of the keys query i sees (schedule.h row_lower).
+    __device__ __forceinline__ int row_lower_of(int, int, int W, int i) const { return row_lower(i, W, 0); }
+    static constexpr bool kDoc = false;
+};
+
+constexpr int kMaxHeadWindows = 64;   // per-head windows travel in the kernel parameters
+
+struct MaskParams {
+    const int* doc_start;      // nullptr: each row is one document
+    int H;
+    int window;                // used when head_windows == 0; <= 0: causal only
+    int head_windows;          // 1: win[bh % H]
+    int win[kMaxHeadWindows];
+    __device__ __forceinline__ int head_window(int bh) const { return head_windows ? win[bh % H] : window; }
+    // Rows past T use the document of the last token.
+    __device__ __forceinline__ int row_lower_of(int bh, int T, int W, int i) const {
+        int d = 0;
+        if (doc_start) d = __ldg(doc_start + (size_t)(bh / H) * T + (i < T ? i : T - 1));
+        return row_lower(i, W, d);
+    }
+    static constexpr bool kDoc = true;
+};
+
+__device__ __forceinline__ int mask_window(const MaskParams& m, int bh) { return m.head_window(bh); }
+__device__ __forceinline__ int mask_row_lower(const MaskParams& m, int bh, int T, int W, int i) {
+    return m.row_lower_of(bh, T, W, i);
+}
+
 struct FwdParams {
     __nv_bfloat16* o;
     float* lse;
@@ -57,7 +93,6 @@ struct FwdParams {
     int n_blocks;         // ceil(n_tiles / 2): 256-query blocks per head
     int heads_per_wave;   // the grid is heads_per_wave * n_blocks CTAs
     int n_waves;          // ceil(BH / heads_per_wave)
-    int window;           // <= 0: causal only
     float scale_log2;     // scale * log2(e)
     uint64_t timeout_ns;
 };
@@ -65,6 +100,13 @@ struct FwdParams {
 // Work item of CTA `cta` in wave `k` (schedule.h).
 __device__ __forceinline__ void fwd_item(const FwdParams& p, int cta, int k, int& bh, int& qb) {
     fwd_item(p.heads_per_wave, p.n_blocks, p.BH, cta, k, bh, qb);
+}
+
+// Key tiles [lo, hi] of query tile qt of head bh with window W.
+template <typename Mask>
+__device__ __forceinline__ void fwd_tile_range(const FwdParams& p, const Mask& m, int bh, int W, int qt, int& lo,
+                                               int& hi) {
+    fwd_key_range_lb(qt, m.row_lower_of(bh, p.T, W, qt * kTile), lo, hi);
 }
 
 template <int D>
@@ -109,11 +151,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-template <int D>
+template <int D, typename Mask>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                const FwdParams p) {
+                const FwdParams p, const __grid_constant__ Mask mask) {
     using C = FwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(smem_align1024(smem_raw));
@@ -183,9 +225,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 int bh, qb;
                 fwd_item(p, cta, k, bh, qb);
                 if (bh < 0) continue;
+                const int W = mask.head_window(bh);
                 int lo0, hi0, lo1, hi1;
-                fwd_key_range(2 * qb, p.window, lo0, hi0);
-                fwd_key_range(2 * qb + 1, p.window, lo1, hi1);
+                fwd_tile_range(p, mask, bh, W, 2 * qb, lo0, hi0);
+                fwd_tile_range(p, mask, bh, W, 2 * qb + 1, lo1, hi1);
                 const int qbuf = n_item % kQBufs;
                 if (n_item >= kQBufs &&
                     !(ok = mbar_wait(&sm.bar_q_empty[qbuf], ((n_item / kQBufs) - 1) & 1, ac)))
@@ -199,6 +242,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const int s = it % kStages;
                     const int n = it / kStages;
                     if (n > 0 && !(ok = mbar_wait(&sm.bar_kv_empty[s], (n - 1) & 1, ac))) break;
+                    if (debug_skip_load(1, it)) continue;         // debug builds: exercise the abort path
                     mbar_arrive_expect_tx(&sm.bar_k[s], kTileBytes);
                     for (int b = 0; b < kBoxes; ++b)
                         tma_load_3d(sm.k[s] + b * 16384, &tm_k, &sm.bar_k[s], b * 64, j * kTile, bh);
@@ -233,9 +277,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 int bh, qb;
                 fwd_item(p, cta, k, bh, qb);
                 if (bh < 0) continue;
+                const int W = mask.head_window(bh);
                 int lo[2], hi[2];
-                fwd_key_range(2 * qb, p.window, lo[0], hi[0]);
-                fwd_key_range(2 * qb + 1, p.window, lo[1], hi[1]);
+                fwd_tile_range(p, mask, bh, W, 2 * qb, lo[0], hi[0]);
+                fwd_tile_range(p, mask, bh, W, 2 * qb + 1, lo[1], hi[1]);
                 const int qbuf = n_item % kQBufs;
                 if (!(ok = mbar_wait(&sm.bar_q[qbuf], (n_item / kQBufs) & 1, ac))) break;
                 const uint32_t q_addr0 = smem_u32(sm.q[qbuf][0]), q_addr1 = smem_u32(sm.q[qbuf][1]);
@@ -277,9 +322,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 int bh, qb;
                 fwd_item(p, cta, k, bh, qb);
                 if (bh < 0) continue;
+                const int W = mask.head_window(bh);
                 int lo0, hi0, lo1, hi1;
-                fwd_key_range(2 * qb, p.window, lo0, hi0);
-                fwd_key_range(2 * qb + 1, p.window, lo1, hi1);
+                fwd_tile_range(p, mask, bh, W, 2 * qb, lo0, hi0);
+                fwd_tile_range(p, mask, bh, W, 2 * qb + 1, lo1, hi1);
                 const int lo = t ? lo1 : lo0, hi = t ? hi1 : hi0;
                 for (int j = lo0; ok && j <= hi1; ++j, ++it) {
                     const int s = it % kStages;
@@ -322,7 +368,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t col_p = t ? C::kColP1 : C::kColP0;
         const uint32_t col_o = t ? C::kColO1 : C::kColO0;
         const float sl2 = p.scale_log2;
-        const int W = p.window;
         bool ok = true;
         int ct = 0;                  // tiles of this warpgroup, over all items
         int n_items = 0;
@@ -333,8 +378,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (bh < 0) continue;
             const int qt = 2 * qb + t;
             const int i_abs = qt * kTile + row;
+            const int W = mask.head_window(bh);
             int lo, hi;
-            fwd_key_range(qt, p.window, lo, hi);
+            fwd_tile_range(p, mask, bh, W, qt, lo, hi);
+            // Visible keys of this row: [row_lo, i_abs].  A key tile needs the per-element mask if
+            // it holds the diagonal or starts before the lower bound of the tile's last row (lower
+            // bounds do not decrease down the tile).
+            const int row_lo = mask.row_lower_of(bh, p.T, W, i_abs);
+            const int last_lo = mask.row_lower_of(bh, p.T, W, qt * kTile + kTile - 1);
             float m_used = -INFINITY;    // reference max of the exponentials (log2 units)
             float l = 0.f;               // running sum of 2^(x - m_used)
             const int n_t = hi - lo + 1;
@@ -357,12 +408,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tc_fence_before();
                     mbar_arrive(&sm.bar_s_free[t]);        // S columns may be overwritten now
                 }
-                const bool need_mask = (j == qt) || (W > 0 && k0 <= qt * kTile + kTile - 1 - W);
+                const bool need_mask = (j == qt) || (k0 < last_lo);
                 if (need_mask) {
                     // Visible columns of this row form one range [c_lo, c_hi]; one unsigned compare
                     // and a select per element, no per-element branch.
                     const int c_hi = i_abs - k0;
-                    const int c_lo = W > 0 ? i_abs - W + 1 - k0 : INT_MIN / 2;
+                    const int c_lo = row_lo - k0;
                     const uint32_t span = (uint32_t)(c_hi - c_lo);
 #pragma unroll
                     for (int e = 0; e < 128; ++e)

@@ -5,12 +5,14 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include <atomic>
 #include <mutex>
 
 #include "attn_bwd.cuh"
 #include "attn_bwd_d64.cuh"
+#include "attn_decode.cuh"
 #include "attn_fwd.cuh"
 #include "gpt_attn.h"
 #include "tmap_cache.h"
@@ -111,9 +113,36 @@ bool set_smem(Kern k, size_t bytes) {
 
 int sm_count();
 
+// Kernel-side mask parameters from the C ABI's description (nullptr: plain causal).  Per-head
+// windows are copied out of the caller's host array into the kernel parameters.
+int make_mask(MaskParams* m, const gpt_attn_mask* a, int H) {
+    memset(m, 0, sizeof(*m));
+    m->H = H;
+    if (!a) return GPT_ATTN_OK;
+    m->window = a->window > 0 ? a->window : 0;
+    m->doc_start = a->doc_start;
+    if (a->doc_start && (reinterpret_cast<uintptr_t>(a->doc_start) & 3u)) return GPT_ATTN_ERR_ALIGN;
+    if (a->head_windows) {
+        if (H > kMaxHeadWindows) return GPT_ATTN_ERR_SHAPE;
+        m->head_windows = 1;
+        for (int h = 0; h < H; ++h) m->win[h] = a->head_windows[h] > 0 ? a->head_windows[h] : 0;
+    }
+    return GPT_ATTN_OK;
+}
+
+// True when every head shares one window and there are no document starts.
+bool plain_window(const MaskParams& m) { return !m.head_windows && !m.doc_start; }
+
+MaskParams window_mask(int window, int H) {
+    gpt_attn_mask a{window, nullptr, nullptr};
+    MaskParams m;
+    make_mask(&m, &a, H);
+    return m;
+}
+
 template <int D>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH, int T, float scale,
-               int window, cudaStream_t st) {
+               const MaskParams& mask, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mo;
     if (!make_tmap_bf16(&mq, q, BH, T, D) || !make_tmap_bf16(&mk, k, BH, T, D) || !make_tmap_bf16(&mv, v, BH, T, D) ||
         !make_tmap_bf16(&mo, o, BH, T, D))
@@ -125,7 +154,6 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.BH = BH;
     p.n_tiles = (T + kTile - 1) / kTile;
     p.n_blocks = (p.n_tiles + 1) / 2;
-    p.window = window > 0 ? window : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = wait_timeout_ns();
     // D = 64: persistent grid, waves of whole heads, heads_per_wave * n_blocks CTAs, at most one
@@ -135,9 +163,15 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     fwd_grid(sm_count(), p.n_blocks, BH, D == 64, p.heads_per_wave, p.n_waves);
     const int hpw = p.heads_per_wave;
     const size_t smem = sizeof(FwdSmem<D>) + 1024;
-    if (!set_smem(attn_fwd_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
     const unsigned grid = (unsigned)((long long)hpw * p.n_blocks);
-    attn_fwd_kernel<D><<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, mo, p);
+    if (plain_window(mask)) {
+        // Causal or one window for every head: the instantiation without per-head or document data.
+        if (!set_smem(attn_fwd_kernel<D, WindowMask>, smem)) return GPT_ATTN_ERR_CUDA;
+        attn_fwd_kernel<D, WindowMask><<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, mo, p, WindowMask{mask.window});
+    } else {
+        if (!set_smem(attn_fwd_kernel<D, MaskParams>, smem)) return GPT_ATTN_ERR_CUDA;
+        attn_fwd_kernel<D, MaskParams><<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, mo, p, mask);
+    }
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
@@ -145,13 +179,16 @@ struct WsLayout {
     float* dq_acc;
     float* lse2;
     float* delta;
+    int* lower2;
+    int* last_qt;
     int* sched;
     int n_tiles;
     int T_pad;
 };
 
 // Workspace: fp32 dQ accumulator [BH, T, D] | lse*log2(e) [BH, T_pad] | Delta [BH, T_pad] |
-// 16 bytes holding the persistent kernel's work-unit counter.
+// row lower bounds [BH, T_pad] and last query tile per key tile [BH, n_tiles] (both used
+// with document masks only) | the persistent kernel's work-unit counter.
 WsLayout ws_layout(void* ws, int BH, int T, int D) {
     WsLayout w;
     w.n_tiles = (T + kTile - 1) / kTile;
@@ -159,7 +196,9 @@ WsLayout ws_layout(void* ws, int BH, int T, int D) {
     w.dq_acc = static_cast<float*>(ws);
     w.lse2 = w.dq_acc + (size_t)BH * T * D;
     w.delta = w.lse2 + (size_t)BH * w.T_pad;
-    w.sched = reinterpret_cast<int*>(w.delta + (size_t)BH * w.T_pad);
+    w.lower2 = reinterpret_cast<int*>(w.delta + (size_t)BH * w.T_pad);
+    w.last_qt = w.lower2 + (size_t)BH * w.T_pad;
+    w.sched = w.last_qt + (size_t)BH * w.n_tiles;
     return w;
 }
 
@@ -178,25 +217,28 @@ int sm_count() {
 }
 
 int launch_bwd_delta(const void* o, const float* lse, const void* dout, int BH, int T, int D, void* ws,
-                     cudaStream_t st) {
+                     const MaskParams& mask, cudaStream_t st) {
     const WsLayout w = ws_layout(ws, BH, T, D);
     const long long rows = (long long)BH * w.T_pad;
     const int rows_per_block = 256 / (D / 8);
     const unsigned grid = (unsigned)((rows + rows_per_block - 1) / rows_per_block);
     const auto* o16 = static_cast<const __nv_bfloat16*>(o);
     const auto* do16 = static_cast<const __nv_bfloat16*>(dout);
+    const bool doc = mask.doc_start != nullptr;
     if (D == 64)
         attn_bwd_prep_kernel<64><<<grid, 256, 0, st>>>(o16, do16, lse, w.lse2, w.delta, w.dq_acc, w.sched, T,
-                                                        w.T_pad, rows);
+                                                        w.T_pad, rows, mask, doc ? w.lower2 : nullptr,
+                                                        w.last_qt, w.n_tiles);
     else
         attn_bwd_prep_kernel<128><<<grid, 256, 0, st>>>(o16, do16, lse, w.lse2, w.delta, w.dq_acc, w.sched, T,
-                                                         w.T_pad, rows);
+                                                         w.T_pad, rows, mask, doc ? w.lower2 : nullptr,
+                                                         w.last_qt, w.n_tiles);
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
 template <int D>
 int launch_bwd_grads(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int BH,
-                     int T, float scale, int window, void* ws, cudaStream_t st) {
+                     int T, float scale, const MaskParams& mask, void* ws, cudaStream_t st) {
     const WsLayout w = ws_layout(ws, BH, T, D);
     CUtensorMap mq, mk, mv, mdo;
     if (!make_tmap_bf16(&mq, q, BH, T, D) || !make_tmap_bf16(&mk, k, BH, T, D) || !make_tmap_bf16(&mv, v, BH, T, D) ||
@@ -213,7 +255,8 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
     p.T_pad = w.T_pad;
     p.BH = BH;
     p.n_tiles = w.n_tiles;
-    p.window = window > 0 ? window : 0;
+    p.lower2 = mask.doc_start ? w.lower2 : nullptr;
+    p.last_qt = mask.doc_start ? w.last_qt : nullptr;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.timeout_ns = wait_timeout_ns();
@@ -225,14 +268,26 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
             !make_tmap_bf16(&mdv, dv, BH, T, D))
             return GPT_ATTN_ERR_CUDA;
         const size_t smem = sizeof(Bwd64Smem) + 1024;
-        if (!set_smem(attn_bwd_kernel, smem)) return GPT_ATTN_ERR_CUDA;
         // persistent: one CTA per SM, work units taken from the counter in the workspace
         const unsigned pgrid = (unsigned)(units < sm_count() ? units : sm_count());
-        attn_bwd_kernel<<<pgrid, kBwd64Threads, smem, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p);
+        if (plain_window(mask)) {
+            if (!set_smem(attn_bwd_kernel<WindowMask>, smem)) return GPT_ATTN_ERR_CUDA;
+            attn_bwd_kernel<WindowMask><<<pgrid, kBwd64Threads, smem, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p,
+                                                                          WindowMask{mask.window});
+        } else {
+            if (!set_smem(attn_bwd_kernel<MaskParams>, smem)) return GPT_ATTN_ERR_CUDA;
+            attn_bwd_kernel<MaskParams><<<pgrid, kBwd64Threads, smem, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p, mask);
+        }
     } else {
         const size_t smem = sizeof(BwdSmem<D>) + 1024;
-        if (!set_smem(attn_bwd_serial_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
-        attn_bwd_serial_kernel<D><<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
+        if (plain_window(mask)) {
+            if (!set_smem(attn_bwd_serial_kernel<D, WindowMask>, smem)) return GPT_ATTN_ERR_CUDA;
+            attn_bwd_serial_kernel<D, WindowMask><<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p,
+                                                                                 WindowMask{mask.window});
+        } else {
+            if (!set_smem(attn_bwd_serial_kernel<D, MaskParams>, smem)) return GPT_ATTN_ERR_CUDA;
+            attn_bwd_serial_kernel<D, MaskParams><<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p, mask);
+        }
     }
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
@@ -249,6 +304,56 @@ int launch_dq_convert(void* dq, int BH, int T, int D, float scale, void* ws, cud
 int check_ws(int B, int H, int T, int D, const void* ws, size_t ws_bytes) {
     if (!ws || ws_bytes < gpt_attn_bwd_workspace_bytes(B, H, T, D)) return GPT_ATTN_ERR_WORKSPACE;
     return misaligned(ws) ? GPT_ATTN_ERR_ALIGN : GPT_ATTN_OK;
+}
+
+// Decode split: aim for two CTAs per SM of a B200 (148 SMs) over all heads, at least 256 keys
+// per split, at most kDecodeMaxChunk.  The same function sizes the workspace and the launch.
+int decode_splits(int BH, int T_max, int window, int* chunk) {
+    const int span = (window > 0 && window < T_max) ? window : T_max;   // keys one query can see
+    int n = (2 * 148 + BH - 1) / BH;
+    const int by_len = (span + 255) / 256;
+    if (n > by_len) n = by_len;
+    if (n < 1) n = 1;
+    if ((span + n - 1) / n > kDecodeMaxChunk) n = (span + kDecodeMaxChunk - 1) / kDecodeMaxChunk;
+    *chunk = (span + n - 1) / n;
+    return n;
+}
+
+int check_decode_shape(int B, int H, int T_max, int D) {
+    if (B < 1 || H < 1 || T_max < 1) return GPT_ATTN_ERR_SHAPE;
+    if (D != 64 && D != 128) return GPT_ATTN_ERR_UNSUPPORTED_D;
+    const long long bh = (long long)B * H;
+    if (bh > 0x7fffffffLL) return GPT_ATTN_ERR_SHAPE;                    // grid x
+    if ((long long)T_max / 256 + 1 > 65535) return GPT_ATTN_ERR_SHAPE;    // splits on grid y
+    if ((long long)T_max > (0x7fffffffffffffffLL / D) / bh) return GPT_ATTN_ERR_SHAPE;
+    return GPT_ATTN_OK;
+}
+
+template <int D>
+int launch_decode(const void* q, const void* k, const void* v, const int* lens, void* o, float* lse, int B, int H,
+                  int T_max, float scale, int window, void* ws, cudaStream_t st) {
+    DecodeParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.k = static_cast<const __nv_bfloat16*>(k);
+    p.v = static_cast<const __nv_bfloat16*>(v);
+    p.lens = lens;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.H = H;
+    p.T_max = T_max;
+    p.window = window > 0 ? window : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const int BH = B * H;
+    p.n_split = decode_splits(BH, T_max, p.window, &p.chunk);
+    p.part_o = static_cast<float*>(ws);
+    p.part_ml = p.part_o + (size_t)BH * p.n_split * D;
+    constexpr int R = kDecodeThreads / (D / 8);
+    const size_t smem = (size_t)(p.chunk > R * D ? p.chunk : R * D) * sizeof(float);
+    if (!set_smem(attn_decode_split_kernel<D>, smem)) return GPT_ATTN_ERR_CUDA;
+    const dim3 grid(BH, p.n_split);
+    attn_decode_split_kernel<D><<<grid, kDecodeThreads, smem, st>>>(p);
+    if (p.n_split > 1) attn_decode_combine_kernel<D><<<BH, D, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
 __global__ void debug_wait_kernel(uint64_t timeout_ns) {
@@ -294,23 +399,31 @@ using namespace gpt_attn;
 
 extern "C" {
 
-int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T, int D,
-                 float scale, int window, void* stream) {
+int gpt_attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T,
+                        int D, float scale, const gpt_attn_mask* mask, void* stream) {
     if (!q || !k || !v || !o || !lse) return GPT_ATTN_ERR_NULL;
-    const int sc = check_shape(B, H, T, D);
+    int sc = check_shape(B, H, T, D);
     if (sc != GPT_ATTN_OK) return sc;
     if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse)) return GPT_ATTN_ERR_ALIGN;
+    MaskParams m;
+    if ((sc = make_mask(&m, mask, H)) != GPT_ATTN_OK) return sc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int BH = B * H;
-    return D == 64 ? launch_fwd<64>(q, k, v, o, lse, BH, T, scale, window, st)
-                   : launch_fwd<128>(q, k, v, o, lse, BH, T, scale, window, st);
+    return D == 64 ? launch_fwd<64>(q, k, v, o, lse, BH, T, scale, m, st)
+                   : launch_fwd<128>(q, k, v, o, lse, BH, T, scale, m, st);
+}
+
+int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T, int D,
+                 float scale, int window, void* stream) {
+    const gpt_attn_mask m{window, nullptr, nullptr};
+    return gpt_attn_fwd_masked(q, k, v, o, lse, B, H, T, D, scale, &m, stream);
 }
 
 size_t gpt_attn_bwd_workspace_bytes(int B, int H, int T, int D) {
     if (check_shape(B, H, T, D) != GPT_ATTN_OK) return 0;
     const size_t bh = (size_t)B * H;
     const size_t t_pad = ((size_t)T + 127) / 128 * 128;
-    return 4 * (bh * T * D + 2 * bh * t_pad) + 16;
+    return 4 * (bh * T * D + 3 * bh * t_pad + bh * (t_pad / 128)) + 16;
 }
 
 int gpt_attn_bwd_delta(const void* o, const float* lse, const void* dO, int B, int H, int T, int D,
@@ -320,7 +433,7 @@ int gpt_attn_bwd_delta(const void* o, const float* lse, const void* dO, int B, i
     if (sc != GPT_ATTN_OK) return sc;
     if ((sc = check_ws(B, H, T, D, workspace, workspace_bytes)) != GPT_ATTN_OK) return sc;
     if (misaligned(o) || misaligned(lse) || misaligned(dO)) return GPT_ATTN_ERR_ALIGN;
-    return launch_bwd_delta(o, lse, dO, B * H, T, D, workspace, static_cast<cudaStream_t>(stream));
+    return launch_bwd_delta(o, lse, dO, B * H, T, D, workspace, window_mask(0, H), static_cast<cudaStream_t>(stream));
 }
 
 int gpt_attn_bwd_grads(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B,
@@ -333,8 +446,9 @@ int gpt_attn_bwd_grads(const void* q, const void* k, const void* v, const void* 
     if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(dO) || misaligned(dk) || misaligned(dv))
         return GPT_ATTN_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return D == 64 ? launch_bwd_grads<64>(q, k, v, dO, dk, dv, B * H, T, scale, window, workspace, st)
-                   : launch_bwd_grads<128>(q, k, v, dO, dk, dv, B * H, T, scale, window, workspace, st);
+    const MaskParams m = window_mask(window, H);
+    return D == 64 ? launch_bwd_grads<64>(q, k, v, dO, dk, dv, B * H, T, scale, m, workspace, st)
+                   : launch_bwd_grads<128>(q, k, v, dO, dk, dv, B * H, T, scale, m, workspace, st);
 }
 
 int gpt_attn_bwd_dq_convert(void* dq, int B, int H, int T, int D, float scale, void* workspace,
@@ -347,9 +461,9 @@ int gpt_attn_bwd_dq_convert(void* dq, int B, int H, int T, int D, float scale, v
     return launch_dq_convert(dq, B * H, T, D, scale, workspace, static_cast<cudaStream_t>(stream));
 }
 
-int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-                 void* dq, void* dk, void* dv, int B, int H, int T, int D, float scale, int window, void* workspace,
-                 size_t workspace_bytes, void* stream) {
+int gpt_attn_bwd_masked(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dO, void* dq, void* dk, void* dv, int B, int H, int T, int D, float scale,
+                        const gpt_attn_mask* mask, void* workspace, size_t workspace_bytes, void* stream) {
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return GPT_ATTN_ERR_NULL;
     int sc = check_shape(B, H, T, D);
     if (sc != GPT_ATTN_OK) return sc;
@@ -357,13 +471,47 @@ int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
     if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse) || misaligned(dO) ||
         misaligned(dq) || misaligned(dk) || misaligned(dv))
         return GPT_ATTN_ERR_ALIGN;
+    MaskParams m;
+    if ((sc = make_mask(&m, mask, H)) != GPT_ATTN_OK) return sc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int BH = B * H;
-    if ((sc = launch_bwd_delta(o, lse, dO, BH, T, D, workspace, st)) != GPT_ATTN_OK) return sc;
-    sc = D == 64 ? launch_bwd_grads<64>(q, k, v, dO, dk, dv, BH, T, scale, window, workspace, st)
-                 : launch_bwd_grads<128>(q, k, v, dO, dk, dv, BH, T, scale, window, workspace, st);
+    if ((sc = launch_bwd_delta(o, lse, dO, BH, T, D, workspace, m, st)) != GPT_ATTN_OK) return sc;
+    sc = D == 64 ? launch_bwd_grads<64>(q, k, v, dO, dk, dv, BH, T, scale, m, workspace, st)
+                 : launch_bwd_grads<128>(q, k, v, dO, dk, dv, BH, T, scale, m, workspace, st);
     if (sc != GPT_ATTN_OK) return sc;
     return launch_dq_convert(dq, BH, T, D, scale, workspace, st);
+}
+
+int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                 void* dq, void* dk, void* dv, int B, int H, int T, int D, float scale, int window, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+    const gpt_attn_mask m{window, nullptr, nullptr};
+    return gpt_attn_bwd_masked(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, &m, workspace, workspace_bytes,
+                               stream);
+}
+
+size_t gpt_attn_decode_workspace_bytes(int B, int H, int T_max, int D, int window) {
+    if (check_decode_shape(B, H, T_max, D) != GPT_ATTN_OK) return 0;
+    int chunk = 0;
+    const int n = decode_splits(B * H, T_max, window > 0 ? window : 0, &chunk);
+    return n > 1 ? (size_t)B * H * n * (D + 2) * sizeof(float) : 16;
+}
+
+int gpt_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* seq_lens, void* o,
+                    float* lse, int B, int H, int T_max, int D, float scale, int window, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+    if (!q || !k_cache || !v_cache || !seq_lens || !o || !lse) return GPT_ATTN_ERR_NULL;
+    const int sc = check_decode_shape(B, H, T_max, D);
+    if (sc != GPT_ATTN_OK) return sc;
+    const size_t need = gpt_attn_decode_workspace_bytes(B, H, T_max, D, window);
+    if (!workspace || workspace_bytes < need) return GPT_ATTN_ERR_WORKSPACE;
+    if (misaligned(q) || misaligned(k_cache) || misaligned(v_cache) || misaligned(o) || misaligned(workspace) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        return GPT_ATTN_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return D == 64 ? launch_decode<64>(q, k_cache, v_cache, seq_lens, o, lse, B, H, T_max, scale, window, workspace, st)
+                   : launch_decode<128>(q, k_cache, v_cache, seq_lens, o, lse, B, H, T_max, scale, window, workspace,
+                                        st);
 }
 
 int gpt_attn_check(void* stream) {
@@ -385,7 +533,9 @@ const char* gpt_attn_status_string(int status) {
         case GPT_ATTN_ERR_ALIGN: return "pointer not 16-byte aligned";
         case GPT_ATTN_ERR_CUDA: return "CUDA error";
         case GPT_ATTN_ERR_TIMEOUT: return "device-side wait timed out";
-        case GPT_ATTN_ERR_WORKSPACE: return "backward workspace missing or too small";
+        case GPT_ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+        case GPT_ATTN_ERR_UNAVAILABLE: return "not available in this build";
+        case GPT_ATTN_ERR_BOUNDS: return "debug build: a kernel bounds check failed";
         default: return "unknown status";
     }
 }
@@ -413,6 +563,17 @@ void gpt_attn_tmap_cache_stats(long long* hits, long long* misses, int* entries)
     if (hits) *hits = h;
     if (misses) *misses = m;
     if (entries) *entries = u;
+}
+
+int gpt_attn_debug_skip_load(int which) {
+#ifdef GPT_ATTN_DEBUG
+    if (which < 0 || which > 2) return GPT_ATTN_ERR_SHAPE;
+    return cudaMemcpyToSymbol(gpt_attn::g_debug_skip, &which, sizeof(int)) == cudaSuccess ? GPT_ATTN_OK
+                                                                                         : GPT_ATTN_ERR_CUDA;
+#else
+    (void)which;
+    return GPT_ATTN_ERR_UNAVAILABLE;
+#endif
 }
 
 int gpt_attn_debug_wait_timeout(int timeout_us, void* stream) {

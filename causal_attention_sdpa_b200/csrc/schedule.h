@@ -17,6 +17,25 @@ namespace gpt_attn {
 
 constexpr int kTile = 128;           // rows per Q tile and per K/V tile
 
+// Lower bound of the keys query i may see: key j is visible iff row_lower(i, ...) <= j <= i.
+// window > 0 keeps the last `window` keys (diagonal included); doc_start_i is the first position
+// of the document holding token i (0 when the row is one document).  Document starts are clamped
+// to [0, i], so every query sees at least itself whatever the input holds.
+GPT_ATTN_HD int row_lower(int i, int window, int doc_start_i) {
+    int lo = window > 0 ? i - window + 1 : 0;
+    int d = doc_start_i < 0 ? 0 : (doc_start_i > i ? i : doc_start_i);
+    if (lo < d) lo = d;
+    return lo < 0 ? 0 : lo;
+}
+
+// Key tiles [lo, hi] hold every key visible to some query of query tile qt, given the lower
+// bound of the tile's first row (lower bounds do not decrease along a row of documents).
+GPT_ATTN_HD void fwd_key_range_lb(int qt, int first_row_lower, int& lo, int& hi) {
+    hi = qt;
+    lo = first_row_lower / kTile;
+    if (lo > hi) lo = hi;
+}
+
 // Key tiles [lo, hi] hold every key visible to some query of query tile qt.
 GPT_ATTN_HD void fwd_key_range(int qt, int window, int& lo, int& hi) {
     hi = qt;
@@ -33,6 +52,18 @@ GPT_ATTN_HD int bwd_last_query_tile(int kt, int n_tiles, int window) {
     const long long last = (long long)kt * kTile + kTile - 1 + window - 1;   // last query seeing the tile
     const long long t = last / kTile;
     return t < n_tiles - 1 ? (int)t : n_tiles - 1;
+}
+
+// Last query tile that sees key tile kt when rows carry lower bounds (document masks):
+// lower_of_tile(qt) is the lower bound of query tile qt's first row.  Lower bounds do not
+// decrease along a row, so tile qt > kt sees the key tile iff its first row's bound is at or
+// before the tile's last key, and those tiles form a prefix [kt, last].
+template <typename LowerOfTile>
+GPT_ATTN_HD int bwd_last_query_tile_lb(int kt, int n_tiles, LowerOfTile lower_of_tile) {
+    const int kend = kt * kTile + kTile - 1;
+    int qt = kt;
+    while (qt + 1 < n_tiles && lower_of_tile(qt + 1) <= kend) ++qt;
+    return qt;
 }
 
 // Forward grid.  A work item is one (head, 256-query block); n_blocks = ceil(n_tiles / 2) per

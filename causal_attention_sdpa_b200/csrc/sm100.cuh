@@ -16,6 +16,32 @@ namespace gpt_attn {
 // is one translation unit, so the definition lives in this header.)
 __device__ int g_status = 0;
 
+#ifdef GPT_ATTN_DEBUG
+// Debug builds: which producer skips one load (see gpt_attn_debug_skip_load), and a bounds check
+// that records GPT_ATTN_ERR_BOUNDS and tells the caller to skip the access.
+__device__ int g_debug_skip = 0;
+__device__ __forceinline__ bool debug_ok(bool cond) {
+    if (!cond) atomicExch(&g_status, GPT_ATTN_ERR_BOUNDS);
+    return cond;
+}
+#define GPT_ATTN_CHECK(cond) \
+    if (!debug_ok(cond)) return
+#else
+#define GPT_ATTN_CHECK(cond)
+#endif
+
+// True in a debug build when the producer of CTA 0 should skip the load of kind `which` (1 forward
+// K/V, 2 backward Q/dO) for its first tile.
+__device__ __forceinline__ bool debug_skip_load(int which, int tile) {
+#ifdef GPT_ATTN_DEBUG
+    return blockIdx.x == 0 && tile == 0 && *(volatile int*)&g_debug_skip == which;
+#else
+    (void)which;
+    (void)tile;
+    return false;
+#endif
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -32,8 +58,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-
-__device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -122,10 +146,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -133,6 +153,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
 
 // 3-D tiled load (no multicast) into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y, int z) {
+    GPT_ATTN_CHECK(x >= 0 && (x & 3) == 0 && z >= 0);
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
@@ -142,6 +163,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
 // 3-D tiled reduce-add shared -> global (element type from the tensor map), no multicast.
 // Coordinates are never negative; rows outside the tensor are skipped by the hardware.
 __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, const void* src, int x, int y, int z) {
+    GPT_ATTN_CHECK(x >= 0 && (x & 3) == 0 && y >= 0 && z >= 0);
     asm volatile(
         "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
         ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
@@ -149,6 +171,7 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, const vo
 }
 // Tile store shared -> global through a tensor map; rows outside the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* src, int x, int y, int z) {
+    GPT_ATTN_CHECK(x >= 0 && (x & 3) == 0 && y >= 0 && z >= 0);
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
                  ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
                  : "memory");
@@ -219,6 +242,7 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 // Each thread of the warp reads 32 consecutive 32-bit columns of its own lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    GPT_ATTN_CHECK((taddr & 0xFFFF) + 32 <= 512 && (taddr >> 16) < 128);
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -258,6 +282,7 @@ __device__ __forceinline__ void tmem_wait_ld_regs2(uint32_t (&a)[32], uint32_t (
 
 // Each thread of the warp writes 16 consecutive 32-bit columns of its own lane.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    GPT_ATTN_CHECK((taddr & 0xFFFF) + 16 <= 512 && (taddr >> 16) < 128);
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
         "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
@@ -268,6 +293,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 
 // Each thread of the warp writes 32 consecutive 32-bit columns of its own lane.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    GPT_ATTN_CHECK((taddr & 0xFFFF) + 32 <= 512 && (taddr >> 16) < 128);
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
         "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
@@ -320,12 +346,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
-}
-
-__device__ __forceinline__ float2 lds_f32x2(uint32_t addr) {
-    float2 v;
-    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
-    return v;
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {

@@ -48,7 +48,9 @@ typedef enum {
     GPT_ATTN_ERR_ALIGN = 4,           /* a pointer is not 16-byte aligned */
     GPT_ATTN_ERR_CUDA = 5,            /* a CUDA call or kernel launch failed */
     GPT_ATTN_ERR_TIMEOUT = 6,         /* a device-side bounded wait ran out */
-    GPT_ATTN_ERR_WORKSPACE = 7        /* backward workspace missing or too small */
+    GPT_ATTN_ERR_WORKSPACE = 7,       /* backward workspace missing or too small */
+    GPT_ATTN_ERR_UNAVAILABLE = 8,     /* not available in this build (debug-only entry points) */
+    GPT_ATTN_ERR_BOUNDS = 9           /* debug build: a kernel's bounds check failed (access skipped) */
 } gpt_attn_status;
 
 /*
@@ -65,12 +67,53 @@ int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int B, int H, int T, int D, float scale, int window, void* stream);
 
 /*
+ * Which keys each query sees, for the *_masked entry points: the long/short
+ * sliding-window pattern and the document-aligned training batches of the
+ * modded-nanogpt README's technique list, in this library's reading.  Key j
+ * is visible to query i of head (b, h) iff
+ *     j <= i,  and  i - j < W_h when W_h >= 1,  and  j >= doc_start[b][i],
+ * where W_h = head_windows[h] if head_windows is given, else `window`
+ * (<= 0 for either means no window), and doc_start[b][i] is the first
+ * position of the document holding token i (0 everywhere when doc_start is
+ * NULL: the row is one document).
+ *   window       : window of every head when head_windows is NULL.
+ *   head_windows : HOST memory, H ints, read during the call (a per-layer
+ *                  pattern is one call per layer with its own window; a
+ *                  window warm-up is a different window per step).  At most
+ *                  64 heads, else GPT_ATTN_ERR_SHAPE.
+ *   doc_start    : DEVICE memory, int32 [B, T], 4-byte aligned, owned by the
+ *                  caller and read by the kernels.  Valid contents: for every
+ *                  row, doc_start[i] <= i, non-decreasing in i, and either
+ *                  doc_start[i] = i (a document starts) or doc_start[i] =
+ *                  doc_start[i-1].  Values are clamped to [0, i], so other
+ *                  contents cannot make a kernel read out of bounds, but give
+ *                  unspecified results.
+ */
+typedef struct {
+    int window;
+    const int* head_windows;
+    const int* doc_start;
+} gpt_attn_mask;
+
+/*
+ * gpt_attn_fwd with the visibility of `mask` (NULL: plain causal).  Same
+ * arguments, layouts and errors as gpt_attn_fwd, plus GPT_ATTN_ERR_SHAPE for
+ * per-head windows with H > 64 and GPT_ATTN_ERR_ALIGN for a doc_start not
+ * 4-byte aligned.  gpt_attn_fwd(..., window, ...) is this call with
+ * {window, NULL, NULL}.
+ */
+int gpt_attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int H, int T, int D, float scale, const gpt_attn_mask* mask,
+                        void* stream);
+
+/*
  * Bytes of device workspace gpt_attn_bwd needs for this shape: an fp32 dQ
- * accumulator [B, H, T, D], two fp32 row vectors per head padded to a
- * multiple of 128 rows (the log2-scaled lse and Delta_i = dO_i . O_i), and
- * 16 bytes for the work-unit counter of the backward kernel:
- * 4 * (B*H*T*D + 2*B*H*T_pad) + 16 with T_pad = ceil(T / 128) * 128.
- * Returns 0 for shapes gpt_attn_bwd would reject.
+ * accumulator [B, H, T, D], three 32-bit row vectors per head padded to a
+ * multiple of 128 rows (the log2-scaled lse, Delta_i = dO_i . O_i, and the
+ * rows' lower key bounds under a document mask), one int per (head, 128-key
+ * tile), and 16 bytes for the work-unit counter of the backward kernel:
+ * 4 * (B*H*T*D + 3*B*H*T_pad + B*H*T_pad/128) + 16 with
+ * T_pad = ceil(T / 128) * 128.  Returns 0 for shapes gpt_attn_bwd would reject.
  */
 size_t gpt_attn_bwd_workspace_bytes(int B, int H, int T, int D);
 
@@ -94,6 +137,17 @@ int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                  const float* lse, const void* dO, void* dq, void* dk, void* dv,
                  int B, int H, int T, int D, float scale, int window,
                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * gpt_attn_bwd with the visibility of `mask` (NULL: plain causal); o and lse
+ * must come from gpt_attn_fwd_masked with the same mask.  Same arguments,
+ * layouts and errors as gpt_attn_bwd and gpt_attn_fwd_masked.  Runs the three
+ * stages below in order (there are no separate masked stage entry points).
+ */
+int gpt_attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                        int B, int H, int T, int D, float scale, const gpt_attn_mask* mask,
+                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * The three stages gpt_attn_bwd runs, in this order, exposed so callers can
@@ -146,6 +200,33 @@ int gpt_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          int B, int H, int T, int D, float scale, int window, void* stream);
 
 /*
+ * Decode attention: one new query per (batch, head) against its cached keys
+ * and values, the inner step of the generation loop of "Un GPT desde cero +
+ * nanoGPT" (Laboratorio L2.1, generate): the model is rerun on the growing
+ * sequence and only the last position is kept, so the result equals the last
+ * row of the causal forward over the sequence so far.  Sequence b holds L_b =
+ * seq_lens[b] tokens (clamped to [0, T_max]) and its query is the last one; it
+ * sees keys j < L_b, and with window >= 1 only j >= L_b - window.
+ *   q            : const bf16 [B, H, D], device (the new token's query).
+ *   k_cache,
+ *   v_cache      : const bf16 [B, H, T_max, D], device; rows >= L_b are not read.
+ *   seq_lens     : const int32 [B], DEVICE memory (so the call can be captured
+ *                  once and replayed as sequences grow), 4-byte aligned.
+ *   o            : bf16 [B, H, D], device, written; lse: fp32 [B, H] (natural
+ *                  log), device, 4-byte aligned.  A sequence with L_b = 0 gets
+ *                  o = 0 and lse = -inf.
+ *   workspace    : device, >= gpt_attn_decode_workspace_bytes(B, H, T_max, D,
+ *                  window) bytes, 16-byte aligned (fp32 partial results of the
+ *                  key splits); contents ignored on entry.
+ * Memory-bound: the caches are read once.  Errors as for gpt_attn_fwd, plus
+ * GPT_ATTN_ERR_WORKSPACE.  Asynchronous on `stream`.
+ */
+size_t gpt_attn_decode_workspace_bytes(int B, int H, int T_max, int D, int window);
+int gpt_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* seq_lens,
+                    void* o, float* lse, int B, int H, int T_max, int D, float scale, int window,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status
  * word: GPT_ATTN_OK, or GPT_ATTN_ERR_TIMEOUT if a kernel's bounded wait ran
  * out since the last check, or GPT_ATTN_ERR_CUDA if a CUDA error is pending.
@@ -165,6 +246,24 @@ const char* gpt_attn_status_string(int status);
  * and the entries held (any pointer may be NULL).  Host only, thread-safe.
  */
 void gpt_attn_tmap_cache_stats(long long* hits, long long* misses, int* entries);
+
+/*
+ * Debug builds only (libgpt_attn_debug.so, compiled with -DGPT_ATTN_DEBUG):
+ * makes the next kernels' producers skip one load, so that the attention
+ * kernels' own bounded waits run out and their abort path is exercised:
+ *   which = 1 : the forward producer of CTA 0 skips its first K/V tile;
+ *   which = 2 : the backward producer of CTA 0 skips its first Q/dO tile;
+ *   which = 0 : no skip (normal operation).
+ * A skipped load is neither issued nor announced to its barrier, so nothing
+ * is left in flight: the consumer's wait runs out after the wait limit
+ * (GPT_ATTN_WAIT_TIMEOUT_MS), every role of the CTA leaves its loop, the
+ * producer waits (bounded) for the loads it did issue, TMEM is released, and
+ * gpt_attn_check reports GPT_ATTN_ERR_TIMEOUT; the context stays usable.
+ * Debug builds also check TMA coordinates and TMEM column ranges before each
+ * access and record GPT_ATTN_ERR_BOUNDS (skipping the access) instead of
+ * issuing a bad one.  Release builds return GPT_ATTN_ERR_UNAVAILABLE.
+ */
+int gpt_attn_debug_skip_load(int which);
 
 /*
  * Diagnostic: launches one small kernel that waits on a shared-memory

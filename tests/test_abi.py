@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_status_strings(L):
-    for code in range(8):
+    for code in range(10):
         s = ga.status_string(code)
         assert s and s != "unknown status"
     assert ga.status_string(99) == "unknown status"
@@ -76,9 +76,10 @@ def test_fwd_misaligned(L, which):
 
 
 def test_workspace_bytes(L):
-    # fp32 dQ accumulator + two fp32 rows per head padded to a multiple of 128 + a 16-byte counter
-    assert ga.gpt_attn_bwd_workspace_bytes(2, 3, 200, 64) == 4 * (6 * 200 * 64 + 2 * 6 * 256) + 16
-    assert ga.gpt_attn_bwd_workspace_bytes(1, 1, 128, 128) == 4 * (128 * 128 + 2 * 128) + 16
+    # fp32 dQ accumulator + three 32-bit rows per head padded to a multiple of 128 + one int per
+    # (head, 128-key tile) + a 16-byte counter
+    assert ga.gpt_attn_bwd_workspace_bytes(2, 3, 200, 64) == 4 * (6 * 200 * 64 + 3 * 6 * 256 + 6 * 2) + 16
+    assert ga.gpt_attn_bwd_workspace_bytes(1, 1, 128, 128) == 4 * (128 * 128 + 3 * 128 + 1) + 16
     assert ga.gpt_attn_bwd_workspace_bytes(1, 1, 8, 32) == 0
     assert ga.gpt_attn_bwd_workspace_bytes(0, 1, 8, 64) == 0
 
@@ -130,3 +131,24 @@ def test_binding_has_no_oracle_dependency():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "oracle.c" not in text and "liboracle" not in text, f
+
+
+def test_masked_entry_point_checks(L):
+    """Mask validation runs before any device work."""
+    vp = ctypes.c_void_p
+    hw = (ctypes.c_int * 65)(*([1] * 65))
+    m = ga.GptAttnMask(0, ctypes.cast(hw, ctypes.POINTER(ctypes.c_int)), None)
+    p = [vp(FAKE)] * 5
+    # per-head windows are limited to 64 heads
+    assert L.gpt_attn_fwd_masked(*p, 1, 65, 8, 64, ctypes.c_float(0.125), ctypes.byref(m), vp(0)) == \
+        ga.GPT_ATTN_ERR_SHAPE
+    # document starts must be 4-byte aligned
+    m2 = ga.GptAttnMask(0, None, FAKE + 2)
+    assert L.gpt_attn_fwd_masked(*p, 1, 2, 8, 64, ctypes.c_float(0.125), ctypes.byref(m2), vp(0)) == \
+        ga.GPT_ATTN_ERR_ALIGN
+    ws = ga.gpt_attn_bwd_workspace_bytes(1, 2, 8, 64)
+    q9 = [vp(FAKE)] * 9
+    assert L.gpt_attn_bwd_masked(*q9, 1, 2, 8, 64, ctypes.c_float(0.125), ctypes.byref(m2), vp(FAKE), ws,
+                                 vp(0)) == ga.GPT_ATTN_ERR_ALIGN
+    assert L.gpt_attn_bwd_masked(*q9[:8], vp(0), 1, 2, 8, 64, ctypes.c_float(0.125), None, vp(FAKE), ws,
+                                 vp(0)) == ga.GPT_ATTN_ERR_NULL

@@ -138,3 +138,58 @@ def test_forward_persistent_order_balances_the_causal_triangle(S):
     # the blocks of one head run in the same wave (shared K/V tiles through L2)
     for b in range(768):
         assert len({items[(b, q)][1] for q in range(4)}) == 1
+
+
+# ---------------------------------------------------------------------------------------------
+# Per-head windows and document starts: the kernels derive tile ranges and mask decisions from
+# each row's lower key bound (row_lower).  Brute force over every (query, key) pair of rows packed
+# with random documents.
+# ---------------------------------------------------------------------------------------------
+def doc_visible(T, window, ds):
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    v = (j <= i) & (j >= np.asarray(ds)[:, None])
+    if window > 0:
+        v &= j > i - window
+    return v
+
+
+def random_doc_starts(T, seed, max_len):
+    import workloads
+    return workloads.make_doc_starts(1, T, seed, max_len)[0]
+
+
+DOC_CASES = [(T, W, L, seed) for T in (1, 100, 128, 300, 1000) for W in (0, 1, 64, 200)
+             for L, seed in ((1, 0), (7, 1), (150, 2), (5000, 3))]
+
+
+@pytest.mark.parametrize("T,W,L,seed", DOC_CASES)
+def test_doc_masks_match_brute_force(S, T, W, L, seed):
+    K = S.sch_tile()
+    n_tiles = -(-T // K)
+    ds = random_doc_starts(T, seed, L).astype(np.int32)
+    vis = doc_visible(T, W, ds)
+    lower = np.array([S.sch_row_lower(i, W, int(ds[i])) for i in range(T)])
+    # each row's lower bound is exactly its first visible key
+    assert (lower == vis.argmax(axis=1)).all()
+    for qt in range(n_tiles):
+        rows = vis[qt * K:(qt + 1) * K]
+        needed = sorted({j // K for j in np.nonzero(rows.any(axis=0))[0]})
+        lo, hi = ctypes.c_int(), ctypes.c_int()
+        S.sch_fwd_key_range_lb(qt, int(lower[qt * K]), ctypes.byref(lo), ctypes.byref(hi))
+        # the forward visits every needed key tile (extra tiles are masked to zero)
+        assert set(needed) <= set(range(lo.value, hi.value + 1)), (qt, lo.value, hi.value, needed)
+        last_lo = lower[min(qt * K + K - 1, T - 1)]
+        for j in range(lo.value, hi.value + 1):
+            full = rows[:, j * K:(j + 1) * K]
+            cols = min(K, T - j * K)
+            unmasked = not (j == qt or j * K < last_lo)
+            if unmasked:   # a tile the kernels do not mask must be fully visible to every row
+                assert full[:, :cols].all(), (qt, j)
+    ptr = ds.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+    for kt in range(n_tiles):
+        cols = vis[:, kt * K:(kt + 1) * K]
+        needed = sorted({i // K for i in np.nonzero(cols.any(axis=1))[0]})
+        last = S.sch_bwd_last_query_tile_lb(kt, n_tiles, T, W, ptr)
+        assert set(needed) <= set(range(kt, last + 1)), (kt, last, needed)
+        assert not needed or needed[-1] == last, (kt, last, needed)
