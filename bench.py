@@ -46,6 +46,8 @@ def parse_args():
                     help="workload number (1-5); the default is the headline shape")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size B (smaller cases for profiler captures)")
     ap.add_argument("--decode", action="store_true",
                     help="time decode attention instead (one new query per sequence against a K/V cache; "
                          "GB/s of cache read against the HBM peak) and print its own JSON line")
@@ -329,6 +331,9 @@ def main():
     if args.decode:
         return run_decode(args)
     w = workloads.BY_INDEX[args.workload]
+    if args.batch is not None:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

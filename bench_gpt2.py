@@ -10,7 +10,9 @@ kernels through their autograd wrapper:
 
   naive     att = softmax(mask(q k^T / sqrt(d))) v, the T x T matrix materialised
   sdpa      torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
-  gpt_attn  causal_attention_sdpa_b200.autograd.gpt_attention(q, k, v)
+  gpt_attn  causal_attention_sdpa_b200.autograd.gpt_attention(q, k, v, out_layout="bthd"): the
+            kernels read q, k, v as strided views of the fused projection and write O in the
+            [B, T, H, D] layout the output projection reads (no transposes)
 
 The model is a plain GPT-2 124M written here (12 layers, 12 heads, d_model 768,
 context 1024, vocabulary padded to 50304, tied embedding and output head, GELU
@@ -62,8 +64,9 @@ class Attention(nn.Module):
         elif self.arm == "sdpa":
             y = F.scaled_dot_product_attention(q, k, v, is_causal=True)
         else:
+            # the head views of the fused projection go in as they are; O comes back token-major
             from causal_attention_sdpa_b200.autograd import gpt_attention
-            y = gpt_attention(q.contiguous(), k.contiguous(), v.contiguous())
+            return self.c_proj(gpt_attention(q, k, v, out_layout="bthd").reshape(B, T, C))
         return self.c_proj(y.transpose(1, 2).reshape(B, T, C))
 
 

@@ -37,8 +37,18 @@ GPT_ATTN_ERR_BOUNDS = 9
 EXPORTED = ("gpt_attn_fwd", "gpt_attn_bwd", "gpt_attn_bwd_workspace_bytes", "gpt_attn_bwd_delta",
             "gpt_attn_bwd_grads", "gpt_attn_bwd_dq_convert", "gpt_attn_check", "gpt_attn_status_string",
             "gpt_attn_debug_wait_timeout", "gpt_attn_bwd_noalloc", "gpt_attn_tmap_cache_stats",
-            "gpt_attn_fwd_masked", "gpt_attn_bwd_masked", "gpt_attn_decode", "gpt_attn_decode_workspace_bytes",
+            "gpt_attn_fwd_ex", "gpt_attn_bwd_ex", "gpt_attn_decode", "gpt_attn_decode_workspace_bytes",
             "gpt_attn_debug_skip_load")
+
+
+class GptAttnStrides(ctypes.Structure):
+    """The C ABI's gpt_attn_strides: element strides (batch, head, token) of a [b, h, t, d] tensor."""
+    _fields_ = [("batch", ctypes.c_longlong), ("head", ctypes.c_longlong), ("token", ctypes.c_longlong)]
+
+
+class GptAttnLayout(ctypes.Structure):
+    """The C ABI's gpt_attn_layout: strides of q, k, v, o, dO, dq, dk, dv."""
+    _fields_ = [(n, GptAttnStrides) for n in ("q", "k", "v", "o", "dO", "dq", "dk", "dv")]
 
 
 class GptAttnMask(ctypes.Structure):
@@ -87,10 +97,11 @@ def lib() -> ctypes.CDLL:
                                                  ctypes.POINTER(ctypes.c_int)]
         L.gpt_attn_tmap_cache_stats.restype = None
         mp = ctypes.POINTER(GptAttnMask)
-        L.gpt_attn_fwd_masked.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, mp, vp]
-        L.gpt_attn_fwd_masked.restype = i
-        L.gpt_attn_bwd_masked.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, mp, vp, sz, vp]
-        L.gpt_attn_bwd_masked.restype = i
+        lp = ctypes.POINTER(GptAttnLayout)
+        L.gpt_attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, mp, lp, vp]
+        L.gpt_attn_fwd_ex.restype = i
+        L.gpt_attn_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, mp, lp, vp, sz, vp]
+        L.gpt_attn_bwd_ex.restype = i
         L.gpt_attn_decode_workspace_bytes.argtypes = [i, i, i, i, i]
         L.gpt_attn_decode_workspace_bytes.restype = sz
         L.gpt_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
@@ -214,48 +225,75 @@ def _mask(H, window=0, head_windows=None, doc_start=None):
     return m, hw
 
 
-def gpt_attn_fwd_masked(q, k, v, scale=None, window=0, head_windows=None, doc_start=None, o=None, lse=None,
-                        stream=None):
-    """Forward pass with per-head windows and/or document starts; returns (o, lse)."""
+def _check_view(name, t, shape):
+    """A bf16 CUDA tensor of the given [B, H, T, D] shape whose last dimension is contiguous."""
+    import torch
+    if t.dtype != torch.bfloat16 or not t.is_cuda or tuple(t.shape) != tuple(shape) or t.stride(3) != 1:
+        raise ValueError(f"{name} must be a CUDA bf16 [B, H, T, D] view of shape {tuple(shape)} with stride 1 in D")
+
+
+def _strides(t):
+    return GptAttnStrides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _layout(**tensors):
+    lay = GptAttnLayout()
+    for n, t in tensors.items():
+        setattr(lay, n, _strides(t))
+    return lay
+
+
+def gpt_attn_fwd_ex(q, k, v, scale=None, window=0, head_windows=None, doc_start=None, o=None, lse=None,
+                    stream=None):
+    """Forward pass with per-head windows and/or document starts, on any [B, H, T, D] views whose D
+    dimension is contiguous (e.g. the q, k, v columns of a fused [B, T, 3, H, D] projection, and an
+    o that is a view of a [B, T, H, D] buffer); returns (o, lse)."""
     import torch
     B, H, T, D = q.shape
     for n, t in (("q", q), ("k", k), ("v", v)):
-        _check_bf16(n, t, q.shape)
+        _check_view(n, t, q.shape)
     if doc_start is not None and tuple(doc_start.shape) != (B, T):
         raise ValueError(f"doc_start must have shape {(B, T)}")
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    o = torch.empty_like(q) if o is None else o
+    o = torch.empty((B, H, T, D), dtype=q.dtype, device=q.device) if o is None else o
+    _check_view("o", o, q.shape)
     lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device) if lse is None else lse
     m, keep = _mask(H, window, head_windows, doc_start)
-    rc = lib().gpt_attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, D, float(scale),
-                                   ctypes.byref(m), _stream_handle(stream))
+    lay = _layout(q=q, k=k, v=v, o=o, dO=o, dq=o, dk=o, dv=o)
+    rc = lib().gpt_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, D, float(scale),
+                               ctypes.byref(m), ctypes.byref(lay), _stream_handle(stream))
     del keep
     if rc != GPT_ATTN_OK:
-        raise GptAttnError(rc, "gpt_attn_fwd_masked")
+        raise GptAttnError(rc, "gpt_attn_fwd_ex")
     return o, lse
 
 
-def gpt_attn_bwd_masked(q, k, v, o, lse, dO, scale=None, window=0, head_windows=None, doc_start=None, dq=None,
-                        dk=None, dv=None, workspace=None, stream=None):
-    """Backward pass under the same mask as gpt_attn_fwd_masked; returns (dq, dk, dv)."""
+def gpt_attn_bwd_ex(q, k, v, o, lse, dO, scale=None, window=0, head_windows=None, doc_start=None, dq=None,
+                    dk=None, dv=None, workspace=None, stream=None):
+    """Backward pass under the same mask as gpt_attn_fwd_ex, on [B, H, T, D] views with contiguous D
+    (dq, dk, dv may be views into one [B, T, 3, H, D] gradient buffer); returns (dq, dk, dv)."""
     import torch
     B, H, T, D = q.shape
     for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dO", dO)):
-        _check_bf16(n, t, q.shape)
+        _check_view(n, t, q.shape)
     if doc_start is not None and tuple(doc_start.shape) != (B, T):
         raise ValueError(f"doc_start must have shape {(B, T)}")
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
+    mk = lambda: torch.empty((B, H, T, D), dtype=q.dtype, device=q.device)
+    dq = mk() if dq is None else dq
+    dk = mk() if dk is None else dk
+    dv = mk() if dv is None else dv
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_view(n, t, q.shape)
     ws, nbytes = _ws(workspace, q)
     m, keep = _mask(H, window, head_windows, doc_start)
-    rc = lib().gpt_attn_bwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk),
-                                   _ptr(dv), B, H, T, D, float(scale), ctypes.byref(m), _ptr(ws), nbytes,
-                                   _stream_handle(stream))
+    lay = _layout(q=q, k=k, v=v, o=o, dO=dO, dq=dq, dk=dk, dv=dv)
+    rc = lib().gpt_attn_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk),
+                               _ptr(dv), B, H, T, D, float(scale), ctypes.byref(m), ctypes.byref(lay), _ptr(ws),
+                               nbytes, _stream_handle(stream))
     del keep
     if rc != GPT_ATTN_OK:
-        raise GptAttnError(rc, "gpt_attn_bwd_masked")
+        raise GptAttnError(rc, "gpt_attn_bwd_ex")
     return dq, dk, dv
 
 

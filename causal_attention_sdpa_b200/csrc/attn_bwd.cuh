@@ -46,6 +46,8 @@ struct BwdParams {
     int* sched;             // work-unit counter of the persistent kernel, zeroed by the prep kernel
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
+    Strides dk_str, dv_str; // dK's and dV's layouts (the D = 128 kernel writes them with plain stores)
+    int H;
     // Document masks only (else nullptr), written by the prep kernel into the workspace:
     const int* lower2;      // [BH, T_pad]   lower bound of each row's visible keys; INT_MAX past T
     const int* last_qt;     // [BH, n_tiles] last query tile that sees each key tile
@@ -117,7 +119,7 @@ attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* _
                      const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ delta,
                      float* __restrict__ dq_acc, int* __restrict__ sched, int T, int T_pad,
                      long long total_rows_pad, const MaskParams mask, int* __restrict__ lower2,
-                     int* __restrict__ last_qt, int n_tiles) {
+                     int* __restrict__ last_qt, int n_tiles, const Strides o_str, const Strides do_str, int H) {
     constexpr int G = D / 8;
     if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0;
     const long long row = (long long)blockIdx.x * (256 / G) + threadIdx.x / G;
@@ -130,8 +132,8 @@ attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* _
     long long src = 0;
     if (valid) {
         src = (bh * T + t) * (long long)D + g * 8;
-        const uint4 a = *reinterpret_cast<const uint4*>(o + src);
-        const uint4 b = *reinterpret_cast<const uint4*>(dout + src);
+        const uint4 a = *reinterpret_cast<const uint4*>(o + o_str.row((int)bh, H, t) + g * 8);
+        const uint4 b = *reinterpret_cast<const uint4*>(dout + do_str.row((int)bh, H, t) + g * 8);
         const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -161,8 +163,10 @@ attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* _
     }
 }
 
+// dQ = bf16(scale * acc): thread i converts 8 consecutive elements of the accumulator [BH, T, D]
+// and writes them to dQ's layout.
 __global__ void attn_dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, long long n8,
-                                       float scale) {
+                                       float scale, int T, int D, int H, const Strides dq_str) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n8) return;
     const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
@@ -172,7 +176,11 @@ __global__ void attn_dq_convert_kernel(const float* __restrict__ acc, __nv_bfloa
     r.y = pack_bf16x2(a.z * scale, a.w * scale);
     r.z = pack_bf16x2(b.x * scale, b.y * scale);
     r.w = pack_bf16x2(b.z * scale, b.w * scale);
-    reinterpret_cast<uint4*>(dq)[i] = r;
+    const long long e = i * 8;                  // first element of the eight
+    const long long row = e / D;
+    const int bh = (int)(row / T);
+    const long long t = row - (long long)bh * T;
+    *reinterpret_cast<uint4*>(dq + dq_str.row(bh, H, t) + (e - row * D)) = r;
 }
 
 template <int D, typename Mask>
@@ -241,10 +249,11 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_do);
+            const int hh = bh % p.H, bb = bh / p.H;
             mbar_arrive_expect_tx(&sm.bar_kv, 2 * kTileBytes);
             for (int b = 0; b < kBoxes; ++b) {
-                tma_load_3d(sm.k + b * 16384, &tm_k, &sm.bar_kv, b * 64, k0, bh);
-                tma_load_3d(sm.v + b * 16384, &tm_v, &sm.bar_kv, b * 64, k0, bh);
+                tma_load_4d(sm.k + b * 16384, &tm_k, &sm.bar_kv, b * 64, k0, hh, bb);
+                tma_load_4d(sm.v + b * 16384, &tm_v, &sm.bar_kv, b * 64, k0, hh, bb);
             }
             int it = 0;
             for (; it < n_q; ++it) {
@@ -254,8 +263,8 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const int q0 = (qt_lo + it) * kTile;
                 mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + (p.lower2 ? 3 : 2) * kTile * 4);
                 for (int b = 0; b < kBoxes; ++b) {
-                    tma_load_3d(sm.q[s] + b * 16384, &tm_q, &sm.bar_qdo_full[s], b * 64, q0, bh);
-                    tma_load_3d(sm.dout[s] + b * 16384, &tm_do, &sm.bar_qdo_full[s], b * 64, q0, bh);
+                    tma_load_4d(sm.q[s] + b * 16384, &tm_q, &sm.bar_qdo_full[s], b * 64, q0, hh, bb);
+                    tma_load_4d(sm.dout[s] + b * 16384, &tm_do, &sm.bar_qdo_full[s], b * 64, q0, hh, bb);
                 }
                 const size_t roff = (size_t)bh * p.T_pad + q0;
                 bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
@@ -420,10 +429,10 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         if (__all_sync(0xffffffffu, ok) && warp_wait(&sm.bar_dkdv_full, 0, ac)) {
             tc_fence_after();
             const bool store = key < p.T;
-            const size_t off = ((size_t)bh * p.T + (store ? key : 0)) * D;
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
-                __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + off;
+                __nv_bfloat16* dst_row = which == 0 ? p.dv + p.dv_str.row(bh, p.H, store ? key : 0)
+                                                    : p.dk + p.dk_str.row(bh, p.H, store ? key : 0);
                 const uint32_t col0 = which == 0 ? C::kColDV : C::kColDK;
                 const float mul = which == 0 ? 1.f : p.scale;     // dK = scale * dS^T Q
 #pragma unroll

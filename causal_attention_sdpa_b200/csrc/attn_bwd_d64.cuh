@@ -175,10 +175,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     };
 
     // Launched with 128 registers per thread (512 x 128 = 65536).  Warpgroup 0
-    // (producer, MMA issuers) 56, the two P/dS warpgroups 184, the dQ
-    // warpgroup 88: 128 x (56 + 184 + 184 + 88) = 65536.
+    // (producer, MMA issuers) 48, the two P/dS warpgroups 184, the dQ
+    // warpgroup 96: 128 x (48 + 184 + 184 + 96) = 65536.
     if (warp < 4) {
-        regs_dec<56>();
+        regs_dec<48>();
         if (warp == 0 && lane == 0) {
             // -------------------------------------------------------- producer
             tma_prefetch_desc(&tm_q);
@@ -199,9 +199,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const Bwd64Unit w = bwd64_unit(u, p, mask);
                 const int kb = n & 1;
                 if (n >= 2 && !(ok = mbar_wait(&sm.bar_kv_empty[kb], ((n >> 1) - 1) & 1, ac))) break;
+                const int hh = w.bh % p.H, bb = w.bh / p.H;
                 mbar_arrive_expect_tx(&sm.bar_kv_full[kb], 2 * kTileBytes);
-                tma_load_3d(sm.k[kb], &tm_k, &sm.bar_kv_full[kb], 0, w.k0, w.bh);
-                tma_load_3d(sm.v[kb], &tm_v, &sm.bar_kv_full[kb], 0, w.k0, w.bh);
+                tma_load_4d(sm.k[kb], &tm_k, &sm.bar_kv_full[kb], 0, w.k0, hh, bb);
+                tma_load_4d(sm.v[kb], &tm_v, &sm.bar_kv_full[kb], 0, w.k0, hh, bb);
                 n_kv = n + 1;
                 for (int i = 0; i < w.n_q; ++i, ++g) {
                     const int s = g % kStages;
@@ -210,8 +211,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (debug_skip_load(2, g)) continue;           // debug builds: exercise the abort path
                     const int q0 = (w.qt_lo + i) * kTile;
                     mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + (p.lower2 ? 3 : 2) * kTile * 4);
-                    tma_load_3d(sm.q[s], &tm_q, &sm.bar_qdo_full[s], 0, q0, w.bh);
-                    tma_load_3d(sm.dout[s], &tm_do, &sm.bar_qdo_full[s], 0, q0, w.bh);
+                    tma_load_4d(sm.q[s], &tm_q, &sm.bar_qdo_full[s], 0, q0, hh, bb);
+                    tma_load_4d(sm.dout[s], &tm_do, &sm.bar_qdo_full[s], 0, q0, hh, bb);
                     const size_t roff = (size_t)w.bh * p.T_pad + q0;
                     bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
                     bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_qdo_full[s]);
@@ -426,7 +427,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
     } else {
-        regs_dec<88>();
+        regs_dec<96>();
         // ------------------------------------------------------------ dQ warpgroup (thread = query / key row)
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
@@ -476,8 +477,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mbar_arrive(&sm.bar_dkdv_staged);
                 if (warp == 12 && lane == 0) {
                     if (!mbar_wait(&sm.bar_dkdv_staged, n & 1, ac)) return false;
-                    tma_store_3d(&tm_dv, sm.v[kb], 0, w.k0, w.bh);
-                    tma_store_3d(&tm_dk, sm.k[kb], 0, w.k0, w.bh);
+                    tma_store_4d(&tm_dv, sm.v[kb], 0, w.k0, w.bh % p.H, w.bh / p.H);
+                    tma_store_4d(&tm_dk, sm.k[kb], 0, w.k0, w.bh % p.H, w.bh / p.H);
                     bulk_commit_group();
                     bulk_wait_group_read0();
                     mbar_arrive(&sm.bar_kv_empty[kb]);

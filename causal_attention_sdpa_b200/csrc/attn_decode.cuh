@@ -79,29 +79,37 @@ attn_decode_split_kernel(const DecodeParams p) {
     const __nv_bfloat16* kh = p.k + (size_t)bh * p.T_max * D;
     const __nv_bfloat16* vh = p.v + (size_t)bh * p.T_max * D;
 
-    // scores: G threads per key row, reduced across the group with shuffles.  Every thread runs
-    // the same number of iterations (rows past the chunk are predicated off), so the whole warp
-    // takes part in every shuffle.
+    // scores: G threads per key row, reduced across the group with shuffles.  Each thread keeps
+    // kU rows in flight (HBM latency is hidden by loads in flight, not by threads alone).  Every
+    // thread runs the same number of iterations (rows past the chunk are predicated off), so the
+    // whole warp takes part in every shuffle.
+    constexpr int kU = 8;
     float mloc = -INFINITY;
-    for (int base = 0; base < n; base += R) {
-        const int jj = base + r;
-        const bool valid = jj < n;
-        float acc = 0.f;
-        if (valid) {
-            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(kh + (size_t)(j0 + jj) * D) + g);
-            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+    for (int base = 0; base < n; base += kU * R) {
+        uint4 raw[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int jj = base + u * R + r;
+            raw[u] = jj < n ? __ldg(reinterpret_cast<const uint4*>(kh + (size_t)(j0 + jj) * D) + g)
+                            : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const uint32_t w4[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+            float acc = 0.f;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
                 acc = fmaf(qv[2 * e], f.x, acc);
                 acc = fmaf(qv[2 * e + 1], f.y, acc);
             }
-        }
 #pragma unroll
-        for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (valid) {
-            if (g == 0) dsm[jj] = acc;
-            mloc = fmaxf(mloc, acc);
+            for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            const int jj = base + u * R + r;
+            if (jj < n) {
+                if (g == 0) dsm[jj] = acc;
+                mloc = fmaxf(mloc, acc);
+            }
         }
     }
     // chunk max over the block
@@ -127,17 +135,30 @@ attn_decode_split_kernel(const DecodeParams p) {
     float l = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecodeThreads / 32; ++w) l += red[w];
-    // o = sum_j p_j V_j: G threads per value row, R rows at once, then a sum over the R groups
+    // o = sum_j p_j V_j: G threads per value row, R rows at once (kV of them in flight per
+    // thread), then a sum over the R groups
+    constexpr int kV = 4;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int jj = r; jj < n; jj += R) {
-        const float pj = dsm[jj];
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(vh + (size_t)(j0 + jj) * D) + g);
-        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+    for (int base = 0; base < n; base += kV * R) {
+        uint4 raw[kV];
+        float pj[kV];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
-            acc[2 * e] = fmaf(pj, f.x, acc[2 * e]);
-            acc[2 * e + 1] = fmaf(pj, f.y, acc[2 * e + 1]);
+        for (int u = 0; u < kV; ++u) {
+            const int jj = base + u * R + r;
+            const bool valid = jj < n;
+            raw[u] = valid ? __ldg(reinterpret_cast<const uint4*>(vh + (size_t)(j0 + jj) * D) + g)
+                           : make_uint4(0u, 0u, 0u, 0u);
+            pj[u] = valid ? dsm[jj] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kV; ++u) {
+            const uint32_t w4[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+                acc[2 * e] = fmaf(pj[u], f.x, acc[2 * e]);
+                acc[2 * e + 1] = fmaf(pj[u], f.y, acc[2 * e + 1]);
+            }
         }
     }
     __syncthreads();                                   // the chunk's probabilities are no longer read

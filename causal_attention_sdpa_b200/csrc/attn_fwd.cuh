@@ -84,9 +84,19 @@ __device__ __forceinline__ int mask_row_lower(const MaskParams& m, int bh, int T
     return m.row_lower_of(bh, T, W, i);
 }
 
+// Element strides of a bf16 tensor indexed [b, h, t, d] (d contiguous).
+struct Strides {
+    long long b, h, t;
+    __host__ __device__ __forceinline__ long long row(int bh, int H, long long t_) const {
+        return (long long)(bh / H) * b + (long long)(bh % H) * h + t_ * t;
+    }
+};
+
 struct FwdParams {
     __nv_bfloat16* o;
     float* lse;
+    Strides o_str;        // O's layout (the D = 128 epilogue writes O with plain stores)
+    int H;
     int T;
     int BH;
     int n_tiles;          // ceil(T / 128)
@@ -233,10 +243,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (n_item >= kQBufs &&
                     !(ok = mbar_wait(&sm.bar_q_empty[qbuf], ((n_item / kQBufs) - 1) & 1, ac)))
                     break;
+                const int hh = bh % p.H, bb = bh / p.H;
                 mbar_arrive_expect_tx(&sm.bar_q[qbuf], 2 * kTileBytes);
                 for (int t = 0; t < 2; ++t)
                     for (int b = 0; b < kBoxes; ++b)
-                        tma_load_3d(sm.q[qbuf][t] + b * 16384, &tm_q, &sm.bar_q[qbuf], b * 64, (2 * qb + t) * kTile, bh);
+                        tma_load_4d(sm.q[qbuf][t] + b * 16384, &tm_q, &sm.bar_q[qbuf], b * 64, (2 * qb + t) * kTile,
+                                    hh, bb);
                 ++n_item;
                 for (int j = lo0; j <= hi1; ++j, ++it) {
                     const int s = it % kStages;
@@ -245,10 +257,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (debug_skip_load(1, it)) continue;         // debug builds: exercise the abort path
                     mbar_arrive_expect_tx(&sm.bar_k[s], kTileBytes);
                     for (int b = 0; b < kBoxes; ++b)
-                        tma_load_3d(sm.k[s] + b * 16384, &tm_k, &sm.bar_k[s], b * 64, j * kTile, bh);
+                        tma_load_4d(sm.k[s] + b * 16384, &tm_k, &sm.bar_k[s], b * 64, j * kTile, hh, bb);
                     mbar_arrive_expect_tx(&sm.bar_v[s], kTileBytes);
                     for (int b = 0; b < kBoxes; ++b)
-                        tma_load_3d(sm.v[s] + b * 16384, &tm_v, &sm.bar_v[s], b * 64, j * kTile, bh);
+                        tma_load_4d(sm.v[s] + b * 16384, &tm_v, &sm.bar_v[s], b * 64, j * kTile, hh, bb);
                 }
             }
             if (sm.abort_flag) {
@@ -552,12 +564,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (!mbar_wait(&sm.bar_ostage_full[t], n_items & 1, ac)) {
                         ok = false;
                     } else if (qt * kTile < p.T) {               // a tile wholly past T stores nothing
-                        tma_store_3d(&tm_o, sm.ostage[t], 0, qt * kTile, bh);
+                        tma_store_4d(&tm_o, sm.ostage[t], 0, qt * kTile, bh % p.H, bh / p.H);
                         bulk_commit_group();
                     }
                 }
             } else {
-                __nv_bfloat16* orow = p.o + ((size_t)bh * p.T + (store ? i_abs : 0)) * D;
+                __nv_bfloat16* orow = p.o + p.o_str.row(bh, p.H, store ? i_abs : 0);
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t r[32];

@@ -53,20 +53,23 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Encodes the tensor map of `key` (see TmapKind): a 3-D view (D, T, BH) of a
-// row-major [BH, T, D] tensor, 128-row boxes whose width is 128 bytes of
-// elements (64 bf16 or 32 fp32 columns), 128-byte swizzle (the UMMA canonical
-// 128B-swizzled layout), zero fill outside the tensor so ragged tails read as zeros.
+// Encodes the tensor map of `key` (see TmapKind): 128-row boxes whose width is 128 bytes of
+// elements (64 bf16 or 32 fp32 columns), 128-byte swizzle (the UMMA canonical 128B-swizzled
+// layout), zero fill outside the tensor so ragged tails read as zeros.  bf16 maps are 4-D
+// (D, T, H, B) with the tensor's own token, head and batch strides, so any [b, h, t, d] view with
+// contiguous d (e.g. the q, k, v columns of a fused [B, T, 3, H, D] projection) is read and
+// written in place; the fp32 accumulator map is 3-D (D, T, B*H), contiguous.
 bool encode_tmap(const TmapKey& key, CUtensorMap* m) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const bool f32 = key.kind == (int)TmapKind::kF32Box32x128;
     const cuuint64_t esz = f32 ? 4 : 2;
-    cuuint64_t dims[3] = {(cuuint64_t)key.d0, (cuuint64_t)key.d1, (cuuint64_t)key.d2};
-    cuuint64_t strides[2] = {(cuuint64_t)key.d0 * esz, (cuuint64_t)key.d1 * key.d0 * esz};
-    cuuint32_t box[3] = {f32 ? 32u : 64u, 128, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+    const cuuint32_t rank = f32 ? 3 : 4;
+    cuuint64_t dims[4] = {(cuuint64_t)key.d0, (cuuint64_t)key.d1, (cuuint64_t)key.d2, (cuuint64_t)key.d3};
+    cuuint64_t strides[3] = {(cuuint64_t)key.s1 * esz, (cuuint64_t)key.s2 * esz, (cuuint64_t)key.s3 * esz};
+    cuuint32_t box[4] = {f32 ? 32u : 64u, 128, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
                     reinterpret_cast<void*>(key.base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -77,19 +80,49 @@ TmapCache<CUtensorMap>& tmap_cache() {
     return c;
 }
 
-bool cached_tmap(CUtensorMap* m, const void* base, TmapKind kind, int BH, int T, int D) {
-    const TmapKey key{reinterpret_cast<uintptr_t>(base), (int)kind, D, T, BH};
+bool cached_tmap(CUtensorMap* m, const TmapKey& key) {
     return tmap_cache().get(key, m, [](const TmapKey& k, CUtensorMap* v) { return encode_tmap(k, v); });
 }
 
-// bf16 [BH, T, D]; 64-column x 128-row boxes.
-bool make_tmap_bf16(CUtensorMap* m, const void* base, int BH, int T, int D) {
-    return cached_tmap(m, base, TmapKind::kBf16Box64x128, BH, T, D);
+// bf16 tensor indexed [b, h, t, d] with strides `st`; 64-column x 128-row boxes.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, int B, int H, int T, int D, const Strides& st) {
+    const TmapKey key{reinterpret_cast<uintptr_t>(base), (int)TmapKind::kBf16Box64x128, D, T, H, B, st.t, st.h, st.b};
+    return cached_tmap(m, key);
 }
 
 // fp32 dQ accumulator [BH, T, D]; 32-column x 128-row boxes for the bulk reduce-add.
 bool make_tmap_f32_acc(CUtensorMap* m, const void* base, int BH, int T, int D) {
-    return cached_tmap(m, base, TmapKind::kF32Box32x128, BH, T, D);
+    const TmapKey key{reinterpret_cast<uintptr_t>(base), (int)TmapKind::kF32Box32x128, D, T, BH, 1,
+                      (long long)D, (long long)T * D, (long long)BH * T * D};
+    return cached_tmap(m, key);
+}
+
+// Strides of every tensor of one call.
+struct Layout {
+    Strides q, k, v, o, dO, dq, dk, dv;
+};
+
+Strides contiguous(int H, int T, int D) { return Strides{(long long)H * T * D, (long long)T * D, (long long)D}; }
+
+Layout contiguous_layout(int H, int T, int D) {
+    const Strides c = contiguous(H, T, D);
+    return Layout{c, c, c, c, c, c, c, c};
+}
+
+// From the C ABI's description (nullptr: contiguous [B, H, T, D]).  TMA needs every stride to be
+// a multiple of 16 bytes (8 elements).
+int make_layout(Layout* L, const gpt_attn_layout* a, int H, int T, int D) {
+    *L = contiguous_layout(H, T, D);
+    if (!a) return GPT_ATTN_OK;
+    const gpt_attn_strides* in[8] = {&a->q, &a->k, &a->v, &a->o, &a->dO, &a->dq, &a->dk, &a->dv};
+    Strides* out[8] = {&L->q, &L->k, &L->v, &L->o, &L->dO, &L->dq, &L->dk, &L->dv};
+    for (int i = 0; i < 8; ++i) {
+        const gpt_attn_strides& x = *in[i];
+        if (x.batch < 0 || x.head < 0 || x.token < 0) return GPT_ATTN_ERR_SHAPE;
+        if ((x.batch | x.head | x.token) & 7) return GPT_ATTN_ERR_ALIGN;
+        *out[i] = Strides{x.batch, x.head, x.token};
+    }
+    return GPT_ATTN_OK;
 }
 
 bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
@@ -141,15 +174,18 @@ MaskParams window_mask(int window, int H) {
 }
 
 template <int D>
-int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH, int T, float scale,
-               const MaskParams& mask, cudaStream_t st) {
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T, float scale,
+               const MaskParams& mask, const Layout& L, cudaStream_t st) {
+    const int BH = B * H;
     CUtensorMap mq, mk, mv, mo;
-    if (!make_tmap_bf16(&mq, q, BH, T, D) || !make_tmap_bf16(&mk, k, BH, T, D) || !make_tmap_bf16(&mv, v, BH, T, D) ||
-        !make_tmap_bf16(&mo, o, BH, T, D))
+    if (!make_tmap_bf16(&mq, q, B, H, T, D, L.q) || !make_tmap_bf16(&mk, k, B, H, T, D, L.k) ||
+        !make_tmap_bf16(&mv, v, B, H, T, D, L.v) || !make_tmap_bf16(&mo, o, B, H, T, D, L.o))
         return GPT_ATTN_ERR_CUDA;
     FwdParams p;
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
+    p.o_str = L.o;
+    p.H = H;
     p.T = T;
     p.BH = BH;
     p.n_tiles = (T + kTile - 1) / kTile;
@@ -216,8 +252,9 @@ int sm_count() {
     return n;
 }
 
-int launch_bwd_delta(const void* o, const float* lse, const void* dout, int BH, int T, int D, void* ws,
-                     const MaskParams& mask, cudaStream_t st) {
+int launch_bwd_delta(const void* o, const float* lse, const void* dout, int B, int H, int T, int D, void* ws,
+                     const MaskParams& mask, const Layout& L, cudaStream_t st) {
+    const int BH = B * H;
     const WsLayout w = ws_layout(ws, BH, T, D);
     const long long rows = (long long)BH * w.T_pad;
     const int rows_per_block = 256 / (D / 8);
@@ -228,21 +265,22 @@ int launch_bwd_delta(const void* o, const float* lse, const void* dout, int BH, 
     if (D == 64)
         attn_bwd_prep_kernel<64><<<grid, 256, 0, st>>>(o16, do16, lse, w.lse2, w.delta, w.dq_acc, w.sched, T,
                                                         w.T_pad, rows, mask, doc ? w.lower2 : nullptr,
-                                                        w.last_qt, w.n_tiles);
+                                                        w.last_qt, w.n_tiles, L.o, L.dO, H);
     else
         attn_bwd_prep_kernel<128><<<grid, 256, 0, st>>>(o16, do16, lse, w.lse2, w.delta, w.dq_acc, w.sched, T,
                                                          w.T_pad, rows, mask, doc ? w.lower2 : nullptr,
-                                                         w.last_qt, w.n_tiles);
+                                                         w.last_qt, w.n_tiles, L.o, L.dO, H);
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
 template <int D>
-int launch_bwd_grads(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int BH,
-                     int T, float scale, const MaskParams& mask, void* ws, cudaStream_t st) {
+int launch_bwd_grads(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv, int B,
+                     int H, int T, float scale, const MaskParams& mask, const Layout& L, void* ws, cudaStream_t st) {
+    const int BH = B * H;
     const WsLayout w = ws_layout(ws, BH, T, D);
     CUtensorMap mq, mk, mv, mdo;
-    if (!make_tmap_bf16(&mq, q, BH, T, D) || !make_tmap_bf16(&mk, k, BH, T, D) || !make_tmap_bf16(&mv, v, BH, T, D) ||
-        !make_tmap_bf16(&mdo, dout, BH, T, D))
+    if (!make_tmap_bf16(&mq, q, B, H, T, D, L.q) || !make_tmap_bf16(&mk, k, B, H, T, D, L.k) ||
+        !make_tmap_bf16(&mv, v, B, H, T, D, L.v) || !make_tmap_bf16(&mdo, dout, B, H, T, D, L.dO))
         return GPT_ATTN_ERR_CUDA;
     BwdParams p;
     p.lse2 = w.lse2;
@@ -251,6 +289,9 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
     p.sched = w.sched;
     p.dk = static_cast<__nv_bfloat16*>(dk);
     p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.dk_str = L.dk;
+    p.dv_str = L.dv;
+    p.H = H;
     p.T = T;
     p.T_pad = w.T_pad;
     p.BH = BH;
@@ -264,8 +305,8 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
     const unsigned grid = (unsigned)units;
     if constexpr (D == 64) {
         CUtensorMap mdq, mdk, mdv;
-        if (!make_tmap_f32_acc(&mdq, w.dq_acc, BH, T, D) || !make_tmap_bf16(&mdk, dk, BH, T, D) ||
-            !make_tmap_bf16(&mdv, dv, BH, T, D))
+        if (!make_tmap_f32_acc(&mdq, w.dq_acc, BH, T, D) || !make_tmap_bf16(&mdk, dk, B, H, T, D, L.dk) ||
+            !make_tmap_bf16(&mdv, dv, B, H, T, D, L.dv))
             return GPT_ATTN_ERR_CUDA;
         const size_t smem = sizeof(Bwd64Smem) + 1024;
         // persistent: one CTA per SM, work units taken from the counter in the workspace
@@ -292,12 +333,13 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
-int launch_dq_convert(void* dq, int BH, int T, int D, float scale, void* ws, cudaStream_t st) {
+int launch_dq_convert(void* dq, int B, int H, int T, int D, float scale, void* ws, const Layout& L, cudaStream_t st) {
+    const int BH = B * H;
     const WsLayout w = ws_layout(ws, BH, T, D);
     const long long n8 = (long long)BH * T * D / 8;
     const int tpb = 256;
     const unsigned grid = (unsigned)((n8 + tpb - 1) / tpb);
-    attn_dq_convert_kernel<<<grid, tpb, 0, st>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq), n8, scale);
+    attn_dq_convert_kernel<<<grid, tpb, 0, st>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq), n8, scale, T, D, H, L.dq);
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
@@ -306,12 +348,12 @@ int check_ws(int B, int H, int T, int D, const void* ws, size_t ws_bytes) {
     return misaligned(ws) ? GPT_ATTN_ERR_ALIGN : GPT_ATTN_OK;
 }
 
-// Decode split: aim for two CTAs per SM of a B200 (148 SMs) over all heads, at least 256 keys
+// Decode split: aim for four CTAs per SM of a B200 (148 SMs) over all heads, at least 64 keys
 // per split, at most kDecodeMaxChunk.  The same function sizes the workspace and the launch.
 int decode_splits(int BH, int T_max, int window, int* chunk) {
     const int span = (window > 0 && window < T_max) ? window : T_max;   // keys one query can see
-    int n = (2 * 148 + BH - 1) / BH;
-    const int by_len = (span + 255) / 256;
+    int n = (4 * 148 + BH - 1) / BH;
+    const int by_len = (span + 63) / 64;
     if (n > by_len) n = by_len;
     if (n < 1) n = 1;
     if ((span + n - 1) / n > kDecodeMaxChunk) n = (span + kDecodeMaxChunk - 1) / kDecodeMaxChunk;
@@ -324,7 +366,7 @@ int check_decode_shape(int B, int H, int T_max, int D) {
     if (D != 64 && D != 128) return GPT_ATTN_ERR_UNSUPPORTED_D;
     const long long bh = (long long)B * H;
     if (bh > 0x7fffffffLL) return GPT_ATTN_ERR_SHAPE;                    // grid x
-    if ((long long)T_max / 256 + 1 > 65535) return GPT_ATTN_ERR_SHAPE;    // splits on grid y
+    if ((long long)T_max / 64 + 1 > 65535) return GPT_ATTN_ERR_SHAPE;     // splits on grid y
     if ((long long)T_max > (0x7fffffffffffffffLL / D) / bh) return GPT_ATTN_ERR_SHAPE;
     return GPT_ATTN_OK;
 }
@@ -399,24 +441,25 @@ using namespace gpt_attn;
 
 extern "C" {
 
-int gpt_attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T,
-                        int D, float scale, const gpt_attn_mask* mask, void* stream) {
+int gpt_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T, int D,
+                    float scale, const gpt_attn_mask* mask, const gpt_attn_layout* layout, void* stream) {
     if (!q || !k || !v || !o || !lse) return GPT_ATTN_ERR_NULL;
     int sc = check_shape(B, H, T, D);
     if (sc != GPT_ATTN_OK) return sc;
     if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(o) || misaligned(lse)) return GPT_ATTN_ERR_ALIGN;
     MaskParams m;
     if ((sc = make_mask(&m, mask, H)) != GPT_ATTN_OK) return sc;
+    Layout L;
+    if ((sc = make_layout(&L, layout, H, T, D)) != GPT_ATTN_OK) return sc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int BH = B * H;
-    return D == 64 ? launch_fwd<64>(q, k, v, o, lse, BH, T, scale, m, st)
-                   : launch_fwd<128>(q, k, v, o, lse, BH, T, scale, m, st);
+    return D == 64 ? launch_fwd<64>(q, k, v, o, lse, B, H, T, scale, m, L, st)
+                   : launch_fwd<128>(q, k, v, o, lse, B, H, T, scale, m, L, st);
 }
 
 int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T, int D,
                  float scale, int window, void* stream) {
     const gpt_attn_mask m{window, nullptr, nullptr};
-    return gpt_attn_fwd_masked(q, k, v, o, lse, B, H, T, D, scale, &m, stream);
+    return gpt_attn_fwd_ex(q, k, v, o, lse, B, H, T, D, scale, &m, nullptr, stream);
 }
 
 size_t gpt_attn_bwd_workspace_bytes(int B, int H, int T, int D) {
@@ -433,7 +476,8 @@ int gpt_attn_bwd_delta(const void* o, const float* lse, const void* dO, int B, i
     if (sc != GPT_ATTN_OK) return sc;
     if ((sc = check_ws(B, H, T, D, workspace, workspace_bytes)) != GPT_ATTN_OK) return sc;
     if (misaligned(o) || misaligned(lse) || misaligned(dO)) return GPT_ATTN_ERR_ALIGN;
-    return launch_bwd_delta(o, lse, dO, B * H, T, D, workspace, window_mask(0, H), static_cast<cudaStream_t>(stream));
+    return launch_bwd_delta(o, lse, dO, B, H, T, D, workspace, window_mask(0, H), contiguous_layout(H, T, D),
+                            static_cast<cudaStream_t>(stream));
 }
 
 int gpt_attn_bwd_grads(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B,
@@ -447,8 +491,9 @@ int gpt_attn_bwd_grads(const void* q, const void* k, const void* v, const void* 
         return GPT_ATTN_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const MaskParams m = window_mask(window, H);
-    return D == 64 ? launch_bwd_grads<64>(q, k, v, dO, dk, dv, B * H, T, scale, m, workspace, st)
-                   : launch_bwd_grads<128>(q, k, v, dO, dk, dv, B * H, T, scale, m, workspace, st);
+    const Layout L = contiguous_layout(H, T, D);
+    return D == 64 ? launch_bwd_grads<64>(q, k, v, dO, dk, dv, B, H, T, scale, m, L, workspace, st)
+                   : launch_bwd_grads<128>(q, k, v, dO, dk, dv, B, H, T, scale, m, L, workspace, st);
 }
 
 int gpt_attn_bwd_dq_convert(void* dq, int B, int H, int T, int D, float scale, void* workspace,
@@ -458,12 +503,13 @@ int gpt_attn_bwd_dq_convert(void* dq, int B, int H, int T, int D, float scale, v
     if (sc != GPT_ATTN_OK) return sc;
     if ((sc = check_ws(B, H, T, D, workspace, workspace_bytes)) != GPT_ATTN_OK) return sc;
     if (misaligned(dq)) return GPT_ATTN_ERR_ALIGN;
-    return launch_dq_convert(dq, B * H, T, D, scale, workspace, static_cast<cudaStream_t>(stream));
+    return launch_dq_convert(dq, B, H, T, D, scale, workspace, contiguous_layout(H, T, D),
+                             static_cast<cudaStream_t>(stream));
 }
 
-int gpt_attn_bwd_masked(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                        const void* dO, void* dq, void* dk, void* dv, int B, int H, int T, int D, float scale,
-                        const gpt_attn_mask* mask, void* workspace, size_t workspace_bytes, void* stream) {
+int gpt_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                    void* dq, void* dk, void* dv, int B, int H, int T, int D, float scale, const gpt_attn_mask* mask,
+                    const gpt_attn_layout* layout, void* workspace, size_t workspace_bytes, void* stream) {
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return GPT_ATTN_ERR_NULL;
     int sc = check_shape(B, H, T, D);
     if (sc != GPT_ATTN_OK) return sc;
@@ -473,21 +519,22 @@ int gpt_attn_bwd_masked(const void* q, const void* k, const void* v, const void*
         return GPT_ATTN_ERR_ALIGN;
     MaskParams m;
     if ((sc = make_mask(&m, mask, H)) != GPT_ATTN_OK) return sc;
+    Layout L;
+    if ((sc = make_layout(&L, layout, H, T, D)) != GPT_ATTN_OK) return sc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int BH = B * H;
-    if ((sc = launch_bwd_delta(o, lse, dO, BH, T, D, workspace, m, st)) != GPT_ATTN_OK) return sc;
-    sc = D == 64 ? launch_bwd_grads<64>(q, k, v, dO, dk, dv, BH, T, scale, m, workspace, st)
-                 : launch_bwd_grads<128>(q, k, v, dO, dk, dv, BH, T, scale, m, workspace, st);
+    if ((sc = launch_bwd_delta(o, lse, dO, B, H, T, D, workspace, m, L, st)) != GPT_ATTN_OK) return sc;
+    sc = D == 64 ? launch_bwd_grads<64>(q, k, v, dO, dk, dv, B, H, T, scale, m, L, workspace, st)
+                 : launch_bwd_grads<128>(q, k, v, dO, dk, dv, B, H, T, scale, m, L, workspace, st);
     if (sc != GPT_ATTN_OK) return sc;
-    return launch_dq_convert(dq, BH, T, D, scale, workspace, st);
+    return launch_dq_convert(dq, B, H, T, D, scale, workspace, L, st);
 }
 
 int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                  void* dq, void* dk, void* dv, int B, int H, int T, int D, float scale, int window, void* workspace,
                  size_t workspace_bytes, void* stream) {
     const gpt_attn_mask m{window, nullptr, nullptr};
-    return gpt_attn_bwd_masked(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, &m, workspace, workspace_bytes,
-                               stream);
+    return gpt_attn_bwd_ex(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, D, scale, &m, nullptr, workspace,
+                           workspace_bytes, stream);
 }
 
 size_t gpt_attn_decode_workspace_bytes(int B, int H, int T_max, int D, int window) {

@@ -1,8 +1,8 @@
 // Host-side cache of encoded TMA tensor maps.
 //
 // A tensor map (CUtensorMap, 128 bytes) is a pure function of its key: the
-// tensor's base address, element type, the 3-D extents (D, T, B*H), the box and
-// the swizzle.  Encoding one costs a driver call; every forward call needs four
+// tensor's base address, element type, extents and strides, the box and the
+// swizzle.  Encoding one costs a driver call; every forward call needs four
 // and every backward call up to seven, so repeated calls on the same buffers
 // (a training loop, a benchmark) look them up here instead.  Because the
 // value depends on nothing but the key, a hit is always correct, even when a
@@ -22,16 +22,18 @@
 namespace gpt_attn {
 
 enum class TmapKind : int {
-    kBf16Box64x128 = 1,    // bf16, 64-column x 128-row boxes, 128-byte swizzle
-    kF32Box32x128 = 2,     // fp32, 32-column x 128-row boxes, 128-byte swizzle
+    kBf16Box64x128 = 1,    // bf16 4-D (D, T, H, B) with strides, 64-column x 128-row boxes, 128-byte swizzle
+    kF32Box32x128 = 2,     // fp32 3-D (D, T, B*H) contiguous, 32-column x 128-row boxes, 128-byte swizzle
 };
 
 struct TmapKey {
     uintptr_t base;
     int kind;
-    int d0, d1, d2;        // extents, innermost first: D, T, B*H
+    int d0, d1, d2, d3;    // extents, innermost first: D, T, H, B (fp32 maps: D, T, B*H, 1)
+    long long s1, s2, s3;  // element strides of dimensions 1..3 (token, head, batch)
     bool operator==(const TmapKey& o) const {
-        return base == o.base && kind == o.kind && d0 == o.d0 && d1 == o.d1 && d2 == o.d2;
+        return base == o.base && kind == o.kind && d0 == o.d0 && d1 == o.d1 && d2 == o.d2 && d3 == o.d3 &&
+               s1 == o.s1 && s2 == o.s2 && s3 == o.s3;
     }
 };
 

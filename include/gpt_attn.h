@@ -67,7 +67,7 @@ int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int B, int H, int T, int D, float scale, int window, void* stream);
 
 /*
- * Which keys each query sees, for the *_masked entry points: the long/short
+ * Which keys each query sees, for the *_ex entry points: the long/short
  * sliding-window pattern and the document-aligned training batches of the
  * modded-nanogpt README's technique list, in this library's reading.  Key j
  * is visible to query i of head (b, h) iff
@@ -96,15 +96,38 @@ typedef struct {
 } gpt_attn_mask;
 
 /*
- * gpt_attn_fwd with the visibility of `mask` (NULL: plain causal).  Same
- * arguments, layouts and errors as gpt_attn_fwd, plus GPT_ATTN_ERR_SHAPE for
- * per-head windows with H > 64 and GPT_ATTN_ERR_ALIGN for a doc_start not
- * 4-byte aligned.  gpt_attn_fwd(..., window, ...) is this call with
- * {window, NULL, NULL}.
+ * Element strides of one bf16 tensor indexed [b, h, t, d] with d contiguous
+ * (stride 1): the address of element (b, h, t, d) is base + b*batch + h*head
+ * + t*token + d.  Contiguous [B, H, T, D] is {H*T*D, T*D, D}; the q, k and v
+ * of a fused projection output [B, T, 3, H, D] are {3*T*H*D, D, 3*H*D} from
+ * base + {0, 1, 2}*H*D ("heads as a batch dimension" without a transpose, as
+ * the GPT-2 lecture's attention module lays them out).  Every stride must be
+ * a multiple of 8 elements (16 bytes, the TMA rule), else GPT_ATTN_ERR_ALIGN;
+ * negative strides give GPT_ATTN_ERR_SHAPE.  Tensors written by a call must
+ * not overlap.
  */
-int gpt_attn_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse,
-                        int B, int H, int T, int D, float scale, const gpt_attn_mask* mask,
-                        void* stream);
+typedef struct {
+    long long batch, head, token;
+} gpt_attn_strides;
+
+/* The layouts of every tensor of a forward or backward call. */
+typedef struct {
+    gpt_attn_strides q, k, v, o;       /* forward and backward */
+    gpt_attn_strides dO, dq, dk, dv;   /* backward only (ignored by the forward) */
+} gpt_attn_layout;
+
+/*
+ * gpt_attn_fwd with the visibility of `mask` (NULL: plain causal) and the
+ * tensor layouts of `layout` (NULL: every tensor contiguous [B, H, T, D]).
+ * Same arguments, ownership and errors as gpt_attn_fwd, plus
+ * GPT_ATTN_ERR_SHAPE for per-head windows with H > 64 and GPT_ATTN_ERR_ALIGN
+ * for a doc_start not 4-byte aligned or a stride not a multiple of 8.  lse
+ * stays contiguous [B, H, T].  gpt_attn_fwd(..., window, ...) is this call
+ * with {window, NULL, NULL} and NULL.
+ */
+int gpt_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int H, int T, int D, float scale, const gpt_attn_mask* mask,
+                    const gpt_attn_layout* layout, void* stream);
 
 /*
  * Bytes of device workspace gpt_attn_bwd needs for this shape: an fp32 dQ
@@ -139,15 +162,17 @@ int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * gpt_attn_bwd with the visibility of `mask` (NULL: plain causal); o and lse
- * must come from gpt_attn_fwd_masked with the same mask.  Same arguments,
- * layouts and errors as gpt_attn_bwd and gpt_attn_fwd_masked.  Runs the three
- * stages below in order (there are no separate masked stage entry points).
+ * gpt_attn_bwd with the visibility of `mask` (NULL: plain causal) and the
+ * layouts of `layout` (NULL: contiguous); o and lse must come from
+ * gpt_attn_fwd_ex with the same mask.  Same arguments and errors as
+ * gpt_attn_bwd and gpt_attn_fwd_ex.  Runs the three stages below in order
+ * (the separate stage entry points take contiguous tensors and a window).
  */
-int gpt_attn_bwd_masked(const void* q, const void* k, const void* v, const void* o,
-                        const float* lse, const void* dO, void* dq, void* dk, void* dv,
-                        int B, int H, int T, int D, float scale, const gpt_attn_mask* mask,
-                        void* workspace, size_t workspace_bytes, void* stream);
+int gpt_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                    const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                    int B, int H, int T, int D, float scale, const gpt_attn_mask* mask,
+                    const gpt_attn_layout* layout, void* workspace, size_t workspace_bytes,
+                    void* stream);
 
 /*
  * The three stages gpt_attn_bwd runs, in this order, exposed so callers can

@@ -140,15 +140,15 @@ def test_masked_entry_point_checks(L):
     m = ga.GptAttnMask(0, ctypes.cast(hw, ctypes.POINTER(ctypes.c_int)), None)
     p = [vp(FAKE)] * 5
     # per-head windows are limited to 64 heads
-    assert L.gpt_attn_fwd_masked(*p, 1, 65, 8, 64, ctypes.c_float(0.125), ctypes.byref(m), vp(0)) == \
+    assert L.gpt_attn_fwd_ex(*p, 1, 65, 8, 64, ctypes.c_float(0.125), ctypes.byref(m), None, vp(0)) == \
         ga.GPT_ATTN_ERR_SHAPE
     # document starts must be 4-byte aligned
     m2 = ga.GptAttnMask(0, None, FAKE + 2)
-    assert L.gpt_attn_fwd_masked(*p, 1, 2, 8, 64, ctypes.c_float(0.125), ctypes.byref(m2), vp(0)) == \
+    assert L.gpt_attn_fwd_ex(*p, 1, 2, 8, 64, ctypes.c_float(0.125), ctypes.byref(m2), None, vp(0)) == \
         ga.GPT_ATTN_ERR_ALIGN
     ws = ga.gpt_attn_bwd_workspace_bytes(1, 2, 8, 64)
     q9 = [vp(FAKE)] * 9
-    assert L.gpt_attn_bwd_masked(*q9, 1, 2, 8, 64, ctypes.c_float(0.125), ctypes.byref(m2), vp(FAKE), ws,
-                                 vp(0)) == ga.GPT_ATTN_ERR_ALIGN
-    assert L.gpt_attn_bwd_masked(*q9[:8], vp(0), 1, 2, 8, 64, ctypes.c_float(0.125), None, vp(FAKE), ws,
-                                 vp(0)) == ga.GPT_ATTN_ERR_NULL
+    assert L.gpt_attn_bwd_ex(*q9, 1, 2, 8, 64, ctypes.c_float(0.125), ctypes.byref(m2), None, vp(FAKE), ws,
+                             vp(0)) == ga.GPT_ATTN_ERR_ALIGN
+    assert L.gpt_attn_bwd_ex(*q9[:8], vp(0), 1, 2, 8, 64, ctypes.c_float(0.125), None, None, vp(FAKE), ws,
+                             vp(0)) == ga.GPT_ATTN_ERR_NULL

@@ -51,6 +51,30 @@ def test_autograd_matches_oracle(B, H, T, D, W):
 
 
 @pytest.mark.gpu
+def test_autograd_strided_inputs_and_token_major_output():
+    """q, k, v as head views of a fused [B, T, 3, H, D] projection, O returned as [B, T, H, D]."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from causal_attention_sdpa_b200 import build
+    build.build()
+    from causal_attention_sdpa_b200.autograd import gpt_attention
+    B, H, T, D = 2, 12, 500, 64
+    q, k, v, do = make_inputs(B, H, T, D, seed=9)
+    qkv = torch.stack([q, k, v], dim=2).permute(0, 3, 2, 1, 4).contiguous().cuda().requires_grad_(True)
+    qs, ks, vs = (qkv[:, :, i].permute(0, 2, 1, 3) for i in range(3))
+    y = gpt_attention(qs, ks, vs, out_layout="bthd")            # [B, T, H, D]
+    assert tuple(y.shape) == (B, T, H, D)
+    y.backward(do.permute(0, 2, 1, 3).cuda())
+    s = 1.0 / math.sqrt(D)
+    ro, _ = oracle.attn_fwd(q, k, v, s)
+    rdq, rdk, rdv, _ = oracle.attn_bwd(q, k, v, do, s)
+    _cmp("o", y.permute(0, 2, 1, 3), ro, TOL_O)
+    g = qkv.grad
+    for i, (name, ref) in enumerate((("dq", rdq), ("dk", rdk), ("dv", rdv))):
+        _cmp(name, g[:, :, i].permute(0, 2, 1, 3), ref, TOL_GRAD)
+
+
+@pytest.mark.gpu
 def test_gpt2_arms_agree():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")

@@ -1,4 +1,4 @@
-"""GPU parity of the masked entry points (gpt_attn_fwd_masked / gpt_attn_bwd_masked) against the
+"""GPU parity of the masked entry points (gpt_attn_fwd_ex / gpt_attn_bwd_ex with a mask) against the
 fp64 oracle's masked functions: per-head windows (the long/short sliding-window pattern) and
 document starts (batches aligned to document ends), from the modded-nanogpt README's technique
 list, on the same seeded inputs, element by element, at the parity tolerances.
@@ -68,8 +68,8 @@ def test_masked_parity(ga, B, H, T, D, hw, W, L, s):
     ds = workloads.make_doc_starts(B, T, seed=T, max_doc_len=L) if L else None
     qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
     dsd = torch.from_numpy(ds).cuda() if ds is not None else None
-    o, lse = ga.gpt_attn_fwd_masked(qd, kd, vd, scale=s, window=W, head_windows=hw, doc_start=dsd)
-    dq, dk, dv = ga.gpt_attn_bwd_masked(qd, kd, vd, o, lse, dod, scale=s, window=W, head_windows=hw,
+    o, lse = ga.gpt_attn_fwd_ex(qd, kd, vd, scale=s, window=W, head_windows=hw, doc_start=dsd)
+    dq, dk, dv = ga.gpt_attn_bwd_ex(qd, kd, vd, o, lse, dod, scale=s, window=W, head_windows=hw,
                                         doc_start=dsd)
     assert ga.gpt_attn_check() == ga.GPT_ATTN_OK
     ro, rl = oracle.attn_fwd_masked(q, k, v, s, hw, W, ds)
@@ -79,12 +79,12 @@ def test_masked_parity(ga, B, H, T, D, hw, W, L, s):
 
 
 def test_plain_entry_points_equal_masked_ones(ga):
-    """gpt_attn_fwd/bwd(window) is gpt_attn_*_masked with {window, NULL, NULL}: same bits."""
+    """gpt_attn_fwd/bwd(window) is gpt_attn_*_ex with {window, NULL, NULL} and no layout: same bits."""
     q, k, v, do = (t.cuda() for t in make_inputs(2, 3, 500, 64, seed=3))
     o1, l1 = ga.gpt_attn_fwd(q, k, v, window=100)
-    o2, l2 = ga.gpt_attn_fwd_masked(q, k, v, window=100)
+    o2, l2 = ga.gpt_attn_fwd_ex(q, k, v, window=100)
     dq1, dk1, dv1 = ga.gpt_attn_bwd(q, k, v, o1, l1, do, window=100)
-    dq2, dk2, dv2 = ga.gpt_attn_bwd_masked(q, k, v, o1, l1, do, window=100)
+    dq2, dk2, dv2 = ga.gpt_attn_bwd_ex(q, k, v, o1, l1, do, window=100)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
@@ -94,6 +94,6 @@ def test_plain_entry_points_equal_masked_ones(ga):
 def test_same_window_per_head_equals_scalar_window(ga):
     q, k, v, _ = (t.cuda() for t in make_inputs(1, 4, 600, 64, seed=4))
     o1, l1 = ga.gpt_attn_fwd(q, k, v, window=200)
-    o2, l2 = ga.gpt_attn_fwd_masked(q, k, v, head_windows=[200] * 4)
+    o2, l2 = ga.gpt_attn_fwd_ex(q, k, v, head_windows=[200] * 4)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)

@@ -66,6 +66,15 @@ def test_every_key_field_separates_entries(C, field):
     assert C.tc_encodes() == 2
 
 
+@pytest.mark.parametrize("which", range(3))
+def test_every_stride_separates_entries(C, which):
+    w0, w1 = ctypes.c_longlong(), ctypes.c_longlong()
+    C.tc_get_stride.argtypes = [ctypes.c_longlong, ctypes.c_int, ctypes.c_longlong, ctypes.POINTER(ctypes.c_longlong)]
+    assert C.tc_get_stride(0x1000, which, 0, ctypes.byref(w0))
+    assert C.tc_get_stride(0x1000, which, 8, ctypes.byref(w1))
+    assert w0.value != w1.value and C.tc_encodes() == 2
+
+
 def test_replacement_keeps_values_correct(C):
     keys = [(0x1000 * (i + 1), 1, 64, 128 * (i + 1), 3) for i in range(7)]   # more keys than slots
     for _ in range(3):
