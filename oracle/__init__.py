@@ -61,6 +61,10 @@ def _load():
         lib.oracle_attn_bwd_masked.restype = ctypes.c_int
         lib.oracle_attn_decode.argtypes = [dp, dp, dp, lp, L, L, L, L, ctypes.c_double, L, dp, dp, ctypes.c_int]
         lib.oracle_attn_decode.restype = ctypes.c_int
+        lib.oracle_qk_prologue_fwd.argtypes = [dp, L, L, L, ctypes.c_int, ctypes.c_double, dp]
+        lib.oracle_qk_prologue_fwd.restype = ctypes.c_int
+        lib.oracle_qk_prologue_bwd.argtypes = [dp, dp, L, L, L, ctypes.c_int, ctypes.c_double, dp]
+        lib.oracle_qk_prologue_bwd.restype = ctypes.c_int
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -182,3 +186,30 @@ def attn_decode(q, k_cache, v_cache, lens, scale: float, window: int = 0, nthrea
     if rc != 0:
         raise RuntimeError(f"oracle_attn_decode failed with code {rc}")
     return o, lse
+
+
+def qk_prologue_fwd(x, norm: bool = True, rope_base: float = 10000.0):
+    """QK-Norm (unit L2 rows) then rotary embedding of half-split pairs by t * base^(-2i/D), on
+    x [..., T, D] (token t = index along T).  rope_base <= 0: no rotation.  Returns fp64."""
+    x = _as_f64(x)
+    *lead, T, D = x.shape
+    NH = int(np.prod(lead)) if lead else 1
+    y = np.zeros_like(x)
+    rc = _load().oracle_qk_prologue_fwd(_ptr(x), NH, T, D, int(bool(norm)), float(rope_base), _ptr(y))
+    if rc != 0:
+        raise RuntimeError(f"oracle_qk_prologue_fwd failed with code {rc}")
+    return y
+
+
+def qk_prologue_bwd(x, dy, norm: bool = True, rope_base: float = 10000.0):
+    """Gradient of qk_prologue_fwd at x for the output gradient dy.  Returns fp64."""
+    x, dy = _as_f64(x), _as_f64(dy)
+    if x.shape != dy.shape:
+        raise ValueError("x and dy must share one shape")
+    *lead, T, D = x.shape
+    NH = int(np.prod(lead)) if lead else 1
+    dx = np.zeros_like(x)
+    rc = _load().oracle_qk_prologue_bwd(_ptr(x), _ptr(dy), NH, T, D, int(bool(norm)), float(rope_base), _ptr(dx))
+    if rc != 0:
+        raise RuntimeError(f"oracle_qk_prologue_bwd failed with code {rc}")
+    return dx

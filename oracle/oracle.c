@@ -281,6 +281,70 @@ int oracle_attn_decode(const double* q, const double* k, const double* v, const 
     return 0;
 }
 
+/* QK-Norm + rotary prologue, the step before attention in the modded-nanogpt README page's
+ * "modernised architecture" item (rotary embeddings, QK-Norm) and the RoPE exercise of "Un GPT
+ * desde cero + nanoGPT".  For each row x (D values) at token position t:
+ *   n = x / max(|x|, 1e-12)                 (QK-Norm: unit L2 norm, no gain)
+ *   y[i]       = n[i] cos a_i - n[i + D/2] sin a_i        i < D/2
+ *   y[i + D/2] = n[i] sin a_i + n[i + D/2] cos a_i        a_i = t * base^(-2i/D)
+ * (each half-split pair is rotated by a_i; norm = 0 skips the normalisation, base <= 0 skips the
+ * rotation).  Rows are [NH, T, D]; head h's token t is row h * T + t. */
+static void prologue_row(const double* x, long D, long t, int norm, double base, double* y, double* nrm) {
+    double ss = 0.0;
+    for (long d = 0; d < D; ++d) ss += x[d] * x[d];
+    double r = sqrt(ss);
+    double inv = 1.0;
+    if (norm) inv = 1.0 / (r > 1e-12 ? r : 1e-12);
+    if (nrm) *nrm = r;
+    const long h = D / 2;
+    for (long i = 0; i < h; ++i) {
+        const double a = base > 0 ? (double)t * pow(base, -2.0 * (double)i / (double)D) : 0.0;
+        const double c = cos(a), s = sin(a);
+        const double x1 = x[i] * inv, x2 = x[i + h] * inv;
+        y[i] = x1 * c - x2 * s;
+        y[i + h] = x1 * s + x2 * c;
+    }
+}
+
+int oracle_qk_prologue_fwd(const double* x, long NH, long T, long D, int norm, double base, double* y) {
+    if (NH < 0 || T < 0 || D <= 0 || (D & 1)) return 1;
+    for (long h = 0; h < NH; ++h)
+        for (long t = 0; t < T; ++t) prologue_row(x + (h * T + t) * D, D, t, norm, base, y + (h * T + t) * D, NULL);
+    return 0;
+}
+
+/* Exact gradient of the prologue: dn = R^T dy (rotate back by a_i), then through the
+ * normalisation dx = (dn - n (n . dn)) / |x| when |x| > 1e-12, else dn / 1e-12. */
+int oracle_qk_prologue_bwd(const double* x, const double* dy, long NH, long T, long D, int norm, double base,
+                           double* dx) {
+    if (NH < 0 || T < 0 || D <= 0 || (D & 1)) return 1;
+    const long hD = D / 2;
+    for (long h = 0; h < NH; ++h)
+        for (long t = 0; t < T; ++t) {
+            const double* xr = x + (h * T + t) * D;
+            const double* g = dy + (h * T + t) * D;
+            double* o = dx + (h * T + t) * D;
+            for (long i = 0; i < hD; ++i) {
+                const double a = base > 0 ? (double)t * pow(base, -2.0 * (double)i / (double)D) : 0.0;
+                const double c = cos(a), s = sin(a);
+                o[i] = g[i] * c + g[i + hD] * s;
+                o[i + hD] = -g[i] * s + g[i + hD] * c;
+            }
+            if (!norm) continue;
+            double ss = 0.0;
+            for (long d = 0; d < D; ++d) ss += xr[d] * xr[d];
+            const double r = sqrt(ss);
+            if (r > 1e-12) {
+                double nd = 0.0;
+                for (long d = 0; d < D; ++d) nd += xr[d] / r * o[d];
+                for (long d = 0; d < D; ++d) o[d] = (o[d] - xr[d] / r * nd) / r;
+            } else {
+                for (long d = 0; d < D; ++d) o[d] /= 1e-12;
+            }
+        }
+    return 0;
+}
+
 int oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
