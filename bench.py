@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--decode", action="store_true",
                     help="time decode attention instead (one new query per sequence against a K/V cache; "
                          "GB/s of cache read against the HBM peak) and print its own JSON line")
+    ap.add_argument("--prologue", action="store_true",
+                    help="time the QK-Norm + rotary prologue (forward and backward) on q and k read from a "
+                         "fused [B, T, 3, H, D] projection and print its own JSON line (GB/s against the HBM peak)")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 256 MB buffer between timed steps (outside their events) and sum the "
                          "per-step times: a cold-L2 figure for workloads whose inputs fit in L2")
@@ -74,11 +77,21 @@ def _code_only(src: str) -> str:
     return re.sub(r"\s+", "", src)
 
 
-def kernel_source_hash() -> str:
-    """Hash of the kernel sources' code (comments and layout excluded), keying recorded ncu data."""
+# Device sources that define each profiled kernel (the file with its body and every header it
+# includes from csrc/).  Host-side launch code is not part of the key; the committed summary
+# records the launch configuration it was captured with.
+KERNEL_SOURCES = {
+    "attn_fwd_kernel": ("attn_fwd.cuh", "schedule.h", "sm100.cuh"),
+    "attn_bwd_kernel": ("attn_bwd_d64.cuh", "attn_bwd.cuh", "attn_fwd.cuh", "schedule.h", "sm100.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str = "attn_bwd_kernel") -> str:
+    """Hash of the code (comments and layout excluded) of the device sources that define `kernel`,
+    keying recorded ncu data: it changes exactly when that kernel's device code does."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "causal_attention_sdpa_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(KERNEL_SOURCES[kernel]):
         with open(os.path.join(csrc, f), encoding="utf-8") as fh:
             h.update(f.encode() + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
@@ -93,7 +106,7 @@ def recorded_traffic(kernel: str, w):
     with open(path) as f:
         d = json.load(f)
     e = d.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or kernel not in KERNEL_SOURCES or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     if (e.get("T"), e.get("D"), e.get("window")) != (w.T, w.D, w.window):
         return None
@@ -326,10 +339,64 @@ def run_decode(args):
                       "cases": lines}), flush=True)
 
 
+def run_prologue(args):
+    """QK-Norm + rotary prologue of q and k (modded-nanogpt's modernised-architecture item) on the
+    long-context shape (B=4 H=6 T=8192 D=128) and on the GPT-2 124M micro-batch-64 shape, inputs
+    read in place from a fused [B, T, 3, H, D] projection.  Memory-bound: bytes that must move per
+    call (forward: q, k read and written; backward: raw q, k and their output gradients read, the
+    raw gradients written) over the call's device time against the HBM peak."""
+    import torch
+    import causal_attention_sdpa_b200 as ga
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    lines = []
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for B, H, T, D in ((4, 6, 8192, 128), (64, 12, 1024, 64)):
+        g = torch.Generator(device=dev)
+        g.manual_seed(99)
+        qkv = torch.randn((B, T, 3, H, D), generator=g, device=dev).to(torch.bfloat16)
+        qr, kr = (qkv[:, :, i].permute(0, 2, 1, 3) for i in range(2))
+        qn, kn = (torch.empty((B, H, T, D), dtype=torch.bfloat16, device=dev) for _ in range(2))
+        dq, dk = (torch.randn((B, H, T, D), generator=g, device=dev).to(torch.bfloat16) for _ in range(2))
+        grad = torch.empty_like(qkv)
+        dqr, dkr = (grad[:, :, i].permute(0, 2, 1, 3) for i in range(2))
+        row_bytes = B * H * T * D * 2
+        calls = {
+            "fwd": (lambda: ga.gpt_attn_qk_prologue_fwd(qr, kr, q_out=qn, k_out=kn), 2 * 2 * row_bytes),
+            "bwd": (lambda: ga.gpt_attn_qk_prologue_bwd(qr, kr, dq, dk, dq_raw=dqr, dk_raw=dkr), 2 * 3 * row_bytes),
+        }
+        case = {"B": B, "H": H, "T": T, "D": D}
+        for name, (fn, nbytes) in calls.items():
+            for _ in range(args.warmup):
+                fn()
+            assert ga.gpt_attn_check() == ga.GPT_ATTN_OK
+            times = []
+            for _ in range(args.steps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+            ms = statistics.median(times)
+            gbs = nbytes / (ms / 1e3) / 1e9
+            case[name] = {"ms": ms, "bytes": nbytes, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
+        lines.append(case)
+    print(json.dumps({"metric": "QK-Norm + rotary prologue bandwidth on 1 B200", "unit": "GB/s",
+                      "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                      "l2": "256 MB written between calls (outside the events)", "steps": args.steps,
+                      "warmup": args.warmup, "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"],
+                      "cases": lines}), flush=True)
+
+
 def main():
     args = parse_args()
     if args.decode:
         return run_decode(args)
+    if args.prologue:
+        return run_prologue(args)
     w = workloads.BY_INDEX[args.workload]
     if args.batch is not None:
         import dataclasses

@@ -38,7 +38,7 @@ EXPORTED = ("gpt_attn_fwd", "gpt_attn_bwd", "gpt_attn_bwd_workspace_bytes", "gpt
             "gpt_attn_bwd_grads", "gpt_attn_bwd_dq_convert", "gpt_attn_check", "gpt_attn_status_string",
             "gpt_attn_debug_wait_timeout", "gpt_attn_bwd_noalloc", "gpt_attn_tmap_cache_stats",
             "gpt_attn_fwd_ex", "gpt_attn_bwd_ex", "gpt_attn_decode", "gpt_attn_decode_workspace_bytes",
-            "gpt_attn_debug_skip_load")
+            "gpt_attn_debug_skip_load", "gpt_attn_qk_prologue_fwd", "gpt_attn_qk_prologue_bwd")
 
 
 class GptAttnStrides(ctypes.Structure):
@@ -106,6 +106,11 @@ def lib() -> ctypes.CDLL:
         L.gpt_attn_decode_workspace_bytes.restype = sz
         L.gpt_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
         L.gpt_attn_decode.restype = i
+        spp = ctypes.POINTER(GptAttnStrides)
+        L.gpt_attn_qk_prologue_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, spp, vp]
+        L.gpt_attn_qk_prologue_fwd.restype = i
+        L.gpt_attn_qk_prologue_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, spp, vp]
+        L.gpt_attn_qk_prologue_bwd.restype = i
         L.gpt_attn_debug_skip_load.argtypes = [i]
         L.gpt_attn_debug_skip_load.restype = i
         L.gpt_attn_debug_wait_timeout.argtypes = [i, vp]
@@ -368,6 +373,44 @@ def gpt_attn_decode(q, k_cache, v_cache, seq_lens, scale=None, window=0, o=None,
     if rc != GPT_ATTN_OK:
         raise GptAttnError(rc, "gpt_attn_decode")
     return o, lse
+
+
+def gpt_attn_qk_prologue_fwd(q_raw, k_raw, qk_norm=True, rope_base=10000.0, q_out=None, k_out=None, stream=None):
+    """QK-Norm + rotary prologue: returns (q, k) bf16 [B, H, T, D] (contiguous unless q_out/k_out are
+    given); q_raw, k_raw may be strided views (e.g. of a fused [B, T, 3, H, D] projection)."""
+    import torch
+    B, H, T, D = q_raw.shape
+    mk = lambda: torch.empty((B, H, T, D), dtype=torch.bfloat16, device=q_raw.device)
+    q_out = mk() if q_out is None else q_out
+    k_out = mk() if k_out is None else k_out
+    ts = [q_raw, k_raw, q_out, k_out]
+    for n, t in zip(("q_raw", "k_raw", "q_out", "k_out"), ts):
+        _check_view(n, t, q_raw.shape)
+    arr = (GptAttnStrides * 4)(*[_strides(t) for t in ts])
+    rc = lib().gpt_attn_qk_prologue_fwd(*[_ptr(t) for t in ts], B, H, T, D, int(bool(qk_norm)), float(rope_base),
+                                        arr, _stream_handle(stream))
+    if rc != GPT_ATTN_OK:
+        raise GptAttnError(rc, "gpt_attn_qk_prologue_fwd")
+    return q_out, k_out
+
+
+def gpt_attn_qk_prologue_bwd(q_raw, k_raw, dq_out, dk_out, qk_norm=True, rope_base=10000.0, dq_raw=None,
+                             dk_raw=None, stream=None):
+    """Gradient of the prologue: returns (dq_raw, dk_raw)."""
+    import torch
+    B, H, T, D = q_raw.shape
+    mk = lambda: torch.empty((B, H, T, D), dtype=torch.bfloat16, device=q_raw.device)
+    dq_raw = mk() if dq_raw is None else dq_raw
+    dk_raw = mk() if dk_raw is None else dk_raw
+    ts = [q_raw, k_raw, dq_out, dk_out, dq_raw, dk_raw]
+    for n, t in zip(("q_raw", "k_raw", "dq_out", "dk_out", "dq_raw", "dk_raw"), ts):
+        _check_view(n, t, q_raw.shape)
+    arr = (GptAttnStrides * 6)(*[_strides(t) for t in ts])
+    rc = lib().gpt_attn_qk_prologue_bwd(*[_ptr(t) for t in ts], B, H, T, D, int(bool(qk_norm)), float(rope_base),
+                                        arr, _stream_handle(stream))
+    if rc != GPT_ATTN_OK:
+        raise GptAttnError(rc, "gpt_attn_qk_prologue_bwd")
+    return dq_raw, dk_raw
 
 
 def gpt_attn_check(stream=None) -> int:

@@ -163,24 +163,26 @@ attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* _
     }
 }
 
-// dQ = bf16(scale * acc): thread i converts 8 consecutive elements of the accumulator [BH, T, D]
-// and writes them to dQ's layout.
-__global__ void attn_dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, long long n8,
-                                       float scale, int T, int D, int H, const Strides dq_str) {
-    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n8) return;
-    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
-    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+// dQ = bf16(scale * acc): G = D / 8 threads per row of the accumulator [BH, T, D], 8 elements
+// (two 16-byte loads, one 16-byte store) each, written to dQ's layout.  One division per thread
+// finds the row's head.
+template <int D>
+__global__ void __launch_bounds__(256)
+attn_dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, long long rows, float scale,
+                       int T, int H, const Strides dq_str) {
+    constexpr int G = D / 8;
+    const long long row = (long long)blockIdx.x * (256 / G) + threadIdx.x / G;
+    if (row >= rows) return;
+    const int g = threadIdx.x % G;
+    const float4 a = reinterpret_cast<const float4*>(acc + row * D)[2 * g];
+    const float4 b = reinterpret_cast<const float4*>(acc + row * D)[2 * g + 1];
     uint4 r;
     r.x = pack_bf16x2(a.x * scale, a.y * scale);
     r.y = pack_bf16x2(a.z * scale, a.w * scale);
     r.z = pack_bf16x2(b.x * scale, b.y * scale);
     r.w = pack_bf16x2(b.z * scale, b.w * scale);
-    const long long e = i * 8;                  // first element of the eight
-    const long long row = e / D;
     const int bh = (int)(row / T);
-    const long long t = row - (long long)bh * T;
-    *reinterpret_cast<uint4*>(dq + dq_str.row(bh, H, t) + (e - row * D)) = r;
+    *reinterpret_cast<uint4*>(dq + dq_str.row(bh, H, row - (long long)bh * T) + g * 8) = r;
 }
 
 template <int D, typename Mask>

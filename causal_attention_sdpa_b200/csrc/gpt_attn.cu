@@ -15,6 +15,7 @@
 #include "attn_decode.cuh"
 #include "attn_fwd.cuh"
 #include "gpt_attn.h"
+#include "qk_prologue.cuh"
 #include "tmap_cache.h"
 
 extern "C" size_t gpt_attn_bwd_workspace_bytes(int B, int H, int T, int D);
@@ -336,10 +337,14 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
 int launch_dq_convert(void* dq, int B, int H, int T, int D, float scale, void* ws, const Layout& L, cudaStream_t st) {
     const int BH = B * H;
     const WsLayout w = ws_layout(ws, BH, T, D);
-    const long long n8 = (long long)BH * T * D / 8;
-    const int tpb = 256;
-    const unsigned grid = (unsigned)((n8 + tpb - 1) / tpb);
-    attn_dq_convert_kernel<<<grid, tpb, 0, st>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq), n8, scale, T, D, H, L.dq);
+    const long long rows = (long long)BH * T;
+    const int rows_per_block = 256 / (D / 8);
+    const unsigned grid = (unsigned)((rows + rows_per_block - 1) / rows_per_block);
+    auto* dq16 = static_cast<__nv_bfloat16*>(dq);
+    if (D == 64)
+        attn_dq_convert_kernel<64><<<grid, 256, 0, st>>>(w.dq_acc, dq16, rows, scale, T, H, L.dq);
+    else
+        attn_dq_convert_kernel<128><<<grid, 256, 0, st>>>(w.dq_acc, dq16, rows, scale, T, H, L.dq);
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
@@ -395,6 +400,35 @@ int launch_decode(const void* q, const void* k, const void* v, const int* lens, 
     const dim3 grid(BH, p.n_split);
     attn_decode_split_kernel<D><<<grid, kDecodeThreads, smem, st>>>(p);
     if (p.n_split > 1) attn_decode_combine_kernel<D><<<BH, D, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
+}
+
+// Strides of n tensors from the C ABI (nullptr: contiguous [B, H, T, D]); same rules as layouts.
+int prologue_strides(Strides* out, const gpt_attn_strides* in, int n, int H, int T, int D) {
+    for (int i = 0; i < n; ++i) {
+        out[i] = contiguous(H, T, D);
+        if (!in) continue;
+        const gpt_attn_strides& x = in[i];
+        if (x.batch < 0 || x.head < 0 || x.token < 0) return GPT_ATTN_ERR_SHAPE;
+        if ((x.batch | x.head | x.token) & 7) return GPT_ATTN_ERR_ALIGN;
+        out[i] = Strides{x.batch, x.head, x.token};
+    }
+    return GPT_ATTN_OK;
+}
+
+int launch_prologue(bool backward, const PrologueParams& p, int D, cudaStream_t st) {
+    // persistent: 2 blocks per SM for each of q and k, all resident at once (4 x 256 threads of
+    // at most 64 registers)
+    const long long rows_per_block = kPrologueThreads / (D / 16);
+    const long long need = (p.rows + rows_per_block - 1) / rows_per_block;
+    const dim3 grid((unsigned)std::min<long long>(need, 2LL * sm_count()), 2);
+    if (backward) {
+        if (D == 64) qk_prologue_bwd_kernel<64><<<grid, 256, 0, st>>>(p);
+        else qk_prologue_bwd_kernel<128><<<grid, 256, 0, st>>>(p);
+    } else {
+        if (D == 64) qk_prologue_fwd_kernel<64><<<grid, 256, 0, st>>>(p);
+        else qk_prologue_fwd_kernel<128><<<grid, 256, 0, st>>>(p);
+    }
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
 }
 
@@ -559,6 +593,55 @@ int gpt_attn_decode(const void* q, const void* k_cache, const void* v_cache, con
     return D == 64 ? launch_decode<64>(q, k_cache, v_cache, seq_lens, o, lse, B, H, T_max, scale, window, workspace, st)
                    : launch_decode<128>(q, k_cache, v_cache, seq_lens, o, lse, B, H, T_max, scale, window, workspace,
                                         st);
+}
+
+int gpt_attn_qk_prologue_fwd(const void* q_raw, const void* k_raw, void* q_out, void* k_out, int B, int H, int T,
+                             int D, int qk_norm, float rope_base, const gpt_attn_strides* strides, void* stream) {
+    if (!q_raw || !k_raw || !q_out || !k_out) return GPT_ATTN_ERR_NULL;
+    int sc = check_shape(B, H, T, D);
+    if (sc != GPT_ATTN_OK) return sc;
+    if (misaligned(q_raw) || misaligned(k_raw) || misaligned(q_out) || misaligned(k_out)) return GPT_ATTN_ERR_ALIGN;
+    Strides st[4];
+    if ((sc = prologue_strides(st, strides, 4, H, T, D)) != GPT_ATTN_OK) return sc;
+    PrologueParams p{};
+    p.x[0] = static_cast<const __nv_bfloat16*>(q_raw);
+    p.x[1] = static_cast<const __nv_bfloat16*>(k_raw);
+    p.out[0] = static_cast<__nv_bfloat16*>(q_out);
+    p.out[1] = static_cast<__nv_bfloat16*>(k_out);
+    p.xs[0] = st[0], p.xs[1] = st[1], p.outs[0] = st[2], p.outs[1] = st[3];
+    p.H = H;
+    p.T = T;
+    p.rows = (long long)B * H * T;
+    p.norm = qk_norm ? 1 : 0;
+    p.base = rope_base;
+    return launch_prologue(false, p, D, static_cast<cudaStream_t>(stream));
+}
+
+int gpt_attn_qk_prologue_bwd(const void* q_raw, const void* k_raw, const void* dq_out, const void* dk_out,
+                             void* dq_raw, void* dk_raw, int B, int H, int T, int D, int qk_norm, float rope_base,
+                             const gpt_attn_strides* strides, void* stream) {
+    if (!q_raw || !k_raw || !dq_out || !dk_out || !dq_raw || !dk_raw) return GPT_ATTN_ERR_NULL;
+    int sc = check_shape(B, H, T, D);
+    if (sc != GPT_ATTN_OK) return sc;
+    if (misaligned(q_raw) || misaligned(k_raw) || misaligned(dq_out) || misaligned(dk_out) || misaligned(dq_raw) ||
+        misaligned(dk_raw))
+        return GPT_ATTN_ERR_ALIGN;
+    Strides st[6];
+    if ((sc = prologue_strides(st, strides, 6, H, T, D)) != GPT_ATTN_OK) return sc;
+    PrologueParams p{};
+    p.x[0] = static_cast<const __nv_bfloat16*>(q_raw);
+    p.x[1] = static_cast<const __nv_bfloat16*>(k_raw);
+    p.dy[0] = static_cast<const __nv_bfloat16*>(dq_out);
+    p.dy[1] = static_cast<const __nv_bfloat16*>(dk_out);
+    p.out[0] = static_cast<__nv_bfloat16*>(dq_raw);
+    p.out[1] = static_cast<__nv_bfloat16*>(dk_raw);
+    p.xs[0] = st[0], p.xs[1] = st[1], p.dys[0] = st[2], p.dys[1] = st[3], p.outs[0] = st[4], p.outs[1] = st[5];
+    p.H = H;
+    p.T = T;
+    p.rows = (long long)B * H * T;
+    p.norm = qk_norm ? 1 : 0;
+    p.base = rope_base;
+    return launch_prologue(true, p, D, static_cast<cudaStream_t>(stream));
 }
 
 int gpt_attn_check(void* stream) {

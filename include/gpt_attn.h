@@ -252,6 +252,37 @@ int gpt_attn_decode(const void* q, const void* k_cache, const void* v_cache, con
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * QK-Norm + rotary prologue of q and k (the step before attention in the
+ * modded-nanogpt README's "modernised architecture" item: rotary embeddings
+ * and QK-Norm; no formulas are given there, this is the reading taken).  For
+ * each row x (D values) of head (b, h) at token t:
+ *     n = x / max(|x|, 1e-12)                    if qk_norm, else n = x
+ *     y[i]       = n[i] cos a_i - n[i + D/2] sin a_i      (i < D/2)
+ *     y[i + D/2] = n[i] sin a_i + n[i + D/2] cos a_i,     a_i = t * rope_base^(-2i/D)
+ * (rope_base <= 1: no rotation).  q_raw, k_raw: const bf16; q_out, k_out:
+ * bf16, written; all [B, H, T, D]-indexed with the strides strides[0..3]
+ * (q_raw, k_raw, q_out, k_out; NULL: all contiguous), e.g. q_raw and k_raw as
+ * the columns of a fused [B, T, 3, H, D] projection and q_out, k_out
+ * contiguous inputs of gpt_attn_fwd.  Memory-bound; fp32 arithmetic.
+ * Errors as for gpt_attn_fwd_ex.  Asynchronous on `stream`.
+ */
+int gpt_attn_qk_prologue_fwd(const void* q_raw, const void* k_raw, void* q_out, void* k_out,
+                             int B, int H, int T, int D, int qk_norm, float rope_base,
+                             const gpt_attn_strides* strides, void* stream);
+
+/*
+ * Gradient of gpt_attn_qk_prologue_fwd: from dq_out, dk_out (the gradients
+ * of q_out, k_out, e.g. from gpt_attn_bwd) and the raw rows, writes
+ * dq_raw, dk_raw: dn = R^T dy (rotated back), then dx = (dn - n (n . dn)) / |x|
+ * under qk_norm.  strides[0..5]: q_raw, k_raw, dq_out, dk_out, dq_raw,
+ * dk_raw (NULL: all contiguous).
+ */
+int gpt_attn_qk_prologue_bwd(const void* q_raw, const void* k_raw, const void* dq_out,
+                             const void* dk_out, void* dq_raw, void* dk_raw, int B, int H, int T,
+                             int D, int qk_norm, float rope_base, const gpt_attn_strides* strides,
+                             void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status
  * word: GPT_ATTN_OK, or GPT_ATTN_ERR_TIMEOUT if a kernel's bounded wait ran
  * out since the last check, or GPT_ATTN_ERR_CUDA if a CUDA error is pending.

@@ -42,14 +42,14 @@ def test_recorded_traffic_is_gated_by_source_hash_and_shape(tmp_path, monkeypatc
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: rec["attn_bwd_kernel"]["source_hash"])
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda k: rec["attn_bwd_kernel"]["source_hash"])
     assert bench.recorded_traffic("attn_bwd_kernel", w3) == pytest.approx(768e6)
     # same T, D, window, fewer heads: scaled by B*H
     assert bench.recorded_traffic("attn_bwd_kernel", workloads.BY_INDEX[2]) == pytest.approx(768e6 * 96 / 768)
     # another shape, another kernel, or changed sources: nothing reported
     assert bench.recorded_traffic("attn_bwd_kernel", workloads.BY_INDEX[5]) is None
     assert bench.recorded_traffic("attn_fwd_kernel", w3) is None
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda k: "0" * 16)
     assert bench.recorded_traffic("attn_bwd_kernel", w3) is None
 
 
@@ -60,11 +60,29 @@ def test_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     dst = tmp_path / "causal_attention_sdpa_b200" / "csrc"
     shutil.copytree(src, dst)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    h0 = bench.kernel_source_hash()
+    h0 = {k: bench.kernel_source_hash(k) for k in bench.KERNEL_SOURCES}
     f = dst / "schedule.h"
     text = f.read_text()
     f.write_text(text.replace("// Key tiles [lo, hi]", "// (reworded)  Key tiles [lo, hi]") + "\n/* note */\n")
-    assert bench.kernel_source_hash() == h0
+    assert {k: bench.kernel_source_hash(k) for k in bench.KERNEL_SOURCES} == h0
     f.write_text(text.replace("constexpr int kTile = 128;", "constexpr int kTile = 64;"))
-    assert bench.kernel_source_hash() != h0
+    for k in bench.KERNEL_SOURCES:
+        assert bench.kernel_source_hash(k) != h0[k]
+    # a change confined to another kernel's file leaves this kernel's key alone
+    f.write_text(text)
+    g = dst / "attn_bwd_d64.cuh"
+    g.write_text(g.read_text().replace("namespace gpt_attn {", "namespace gpt_attn {\nconstexpr int kUnused = 1;", 1))
+    assert bench.kernel_source_hash("attn_fwd_kernel") == h0["attn_fwd_kernel"]
+    assert bench.kernel_source_hash("attn_bwd_kernel") != h0["attn_bwd_kernel"]
 
+
+def test_kernel_sources_cover_the_kernels_includes():
+    """Every csrc/ header that a profiled kernel's files include is part of its hash key."""
+    import re
+    csrc = os.path.join(ROOT, "causal_attention_sdpa_b200", "csrc")
+    for kernel, files in bench.KERNEL_SOURCES.items():
+        for f in files:
+            text = open(os.path.join(csrc, f), encoding="utf-8").read()
+            for inc in re.findall(r'#include "([^"]+)"', text):
+                if os.path.exists(os.path.join(csrc, inc)):
+                    assert inc in files, (kernel, f, inc)
