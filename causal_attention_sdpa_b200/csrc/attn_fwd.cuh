@@ -342,7 +342,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int j = lo0; ok && j <= hi1; ++j, ++it) {
                     const int s = it % kStages;
                     if (j < lo || j > hi) {
-                        mbar_arrive(&sm.bar_kv_empty[s]);   // nothing of this warp reads stage s here
+                        // Nothing of this warp reads stage s here.  Arrive only once the stage holds
+                        // this tile: an arrival made earlier could complete the stage's previous phase
+                        // while another warp's MMAs still read it.
+                        if (!(ok = mbar_wait(&sm.bar_k[s], (it / kStages) & 1, ac))) break;
+                        mbar_arrive(&sm.bar_kv_empty[s]);
                         continue;
                     }
                     const int i = j - lo;

@@ -612,6 +612,7 @@ int gpt_attn_qk_prologue_fwd(const void* q_raw, const void* k_raw, void* q_out, 
     p.H = H;
     p.T = T;
     p.rows = (long long)B * H * T;
+    p.token_major = st[0].t < st[0].h ? 1 : 0;    // walk rows in q_raw's memory order
     p.norm = qk_norm ? 1 : 0;
     p.base = rope_base;
     return launch_prologue(false, p, D, static_cast<cudaStream_t>(stream));
@@ -639,6 +640,7 @@ int gpt_attn_qk_prologue_bwd(const void* q_raw, const void* k_raw, const void* d
     p.H = H;
     p.T = T;
     p.rows = (long long)B * H * T;
+    p.token_major = st[0].t < st[0].h ? 1 : 0;    // walk rows in q_raw's memory order
     p.norm = qk_norm ? 1 : 0;
     p.base = rope_base;
     return launch_prologue(true, p, D, static_cast<cudaStream_t>(stream));

@@ -32,12 +32,29 @@ struct PrologueParams {
     long long rows;                // B * H * T per tensor
     int norm;                      // 1: QK-Norm
     float base;                    // rope base; <= 1: no rotation
+    int token_major;               // 1: rows in (b, t, h) order, else (b, h, t)
 };
+
+// Head and token of linear row `row`.  Rows are walked in the order of the input's memory: for
+// q and k read out of a fused [B, T, 3, H, D] projection the heads of one token are adjacent
+// ((b, t, h) order), for a [B, H, T, D] tensor the tokens of one head ((b, h, t) order), so the
+// rows that all blocks handle at one time cover a dense stretch of memory.
+__device__ __forceinline__ void prologue_row(const PrologueParams& p, long long row, int& bh, int& t) {
+    if (p.token_major) {
+        const long long bt = row / p.H;              // b * T + t
+        const int h = (int)(row - bt * p.H);
+        const int b = (int)(bt / p.T);
+        t = (int)(bt - (long long)b * p.T);
+        bh = b * p.H + h;
+    } else {
+        bh = (int)(row / p.T);
+        t = (int)(row - (long long)bh * p.T);
+    }
+}
 
 constexpr int kPrologueThreads = 256;
 
-__device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* p, float (&f)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
+__device__ __forceinline__ void unpack_bf16x8(const uint4 u, float (&f)[8]) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -45,6 +62,10 @@ __device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* p, float (&f)[8
         f[2 * e] = t.x;
         f[2 * e + 1] = t.y;
     }
+}
+
+__device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* p, float (&f)[8]) {
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(p), f);
 }
 
 __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* p, const float (&f)[8]) {
@@ -68,15 +89,17 @@ __device__ __forceinline__ void prologue_rev_per_token(float base, double* rev) 
     __syncthreads();
 }
 
-// cos and sin of the angles of pairs 8j .. 8j + 7 at token t, each angle first reduced to
-// [-pi, pi] in fp64.
+// cos and sin of t * 2 pi * rev, the angle first reduced to [-pi, pi] in fp64.
+__device__ __forceinline__ void prologue_angle(int t, double rev, float& c, float& s) {
+    const double r = (double)t * rev;
+    const float a = (float)(r - rint(r)) * 6.283185307179586f;
+    __sincosf(a, &s, &c);
+}
+
+// The same for the angles of pairs 8j .. 8j + 7 at token t (rev points at pair 8j).
 __device__ __forceinline__ void prologue_angles(int t, const double* rev, float (&c)[8], float (&s)[8]) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const double r = (double)t * rev[e];
-        const float a = (float)(r - rint(r)) * 6.283185307179586f;
-        __sincosf(a, &s[e], &c[e]);
-    }
+    for (int e = 0; e < 8; ++e) prologue_angle(t, rev[e], c[e], s[e]);
 }
 
 // Sum over the G lanes of a row's group (G a power of two, groups aligned within the warp).
@@ -88,9 +111,10 @@ __device__ __forceinline__ float group_sum(float v) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPrologueThreads)
+__global__ void __launch_bounds__(kPrologueThreads, 4)
 qk_prologue_fwd_kernel(const PrologueParams p) {
     constexpr int G = D / 16, H2 = D / 2, kRows = kPrologueThreads / G;
+    constexpr int U = 2;                             // rows per lane group and iteration
     const int which = blockIdx.y;                    // 0: q, 1: k
     const int j = threadIdx.x % G;
     __shared__ double rev[D / 2];
@@ -98,40 +122,57 @@ qk_prologue_fwd_kernel(const PrologueParams p) {
     const __nv_bfloat16* xb = p.x[which];
     __nv_bfloat16* yb = p.out[which];
     const Strides xs = p.xs[which], ys = p.outs[which];
-    // Rows advance in steps of the whole grid.  The loop bound is taken on the warp's first row,
-    // so every lane of a warp runs the same iterations and takes part in every shuffle; lanes whose
+    const long long stride = (long long)gridDim.x * kRows;
+    // Each iteration takes U rows a grid stride apart, all loads issued before any arithmetic, so
+    // 4 x 16 bytes per lane are in flight.  The loop bound is taken on the warp's first row, so
+    // every lane of a warp runs the same iterations and takes part in every shuffle; lanes whose
     // row is past the end compute on zeros and store nothing.
     for (long long row0 = (long long)blockIdx.x * kRows + (threadIdx.x & ~31) / G; row0 < p.rows;
-         row0 += (long long)gridDim.x * kRows) {
-        const long long row = row0 + (threadIdx.x & 31) / G;
-        const bool valid = row < p.rows;
-        const int bh = valid ? (int)(row / p.T) : 0;
-        const int t = valid ? (int)(row - (long long)bh * p.T) : 0;
-        const __nv_bfloat16* x = xb + xs.row(bh, p.H, t) + 8 * j;
-        float a[8] = {}, b[8] = {};                  // elements 8j + e and D/2 + 8j + e
-        if (valid) {
-            load_bf16x8(x, a);
-            load_bf16x8(x + H2, b);
-        }
-        float inv = 1.f;
-        if (p.norm) {
-            float ss = 0.f;
+         row0 += U * stride) {
+        bool valid[U];
+        int bh[U], t[U];
+        uint4 ra[U], rb[U];                          // elements 8j + e and D/2 + 8j + e, still bf16
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ss = fmaf(a[e], a[e], fmaf(b[e], b[e], ss));
-            inv = 1.f / fmaxf(sqrtf(group_sum<G>(ss)), 1e-12f);
+        for (int u = 0; u < U; ++u) {
+            const long long row = row0 + u * stride + (threadIdx.x & 31) / G;
+            valid[u] = row < p.rows;
+            bh[u] = 0, t[u] = 0;
+            if (valid[u]) prologue_row(p, row, bh[u], t[u]);
+            ra[u] = rb[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (valid[u]) {
+                const __nv_bfloat16* x = xb + xs.row(bh[u], p.H, t[u]) + 8 * j;
+                ra[u] = *reinterpret_cast<const uint4*>(x);
+                rb[u] = *reinterpret_cast<const uint4*>(x + H2);
+            }
         }
-        float c[8], s[8], ya[8], yb2[8];
-        prologue_angles(t, rev + 8 * j, c, s);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float u = a[e] * inv, w = b[e] * inv;
-            ya[e] = u * c[e] - w * s[e];
-            yb2[e] = u * s[e] + w * c[e];
-        }
-        if (valid) {
-            __nv_bfloat16* y = yb + ys.row(bh, p.H, t) + 8 * j;
-            store_bf16x8(y, ya);
-            store_bf16x8(y + H2, yb2);
+        for (int u = 0; u < U; ++u) {
+            float a[8], b[8];
+            unpack_bf16x8(ra[u], a);
+            unpack_bf16x8(rb[u], b);
+            float inv = 1.f;
+            if (p.norm) {
+                float ss = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss = fmaf(a[e], a[e], fmaf(b[e], b[e], ss));
+                inv = 1.f / fmaxf(sqrtf(group_sum<G>(ss)), 1e-12f);
+            }
+            // rotate pair by pair, packing the outputs as they are produced
+            uint32_t oa[4], ob[4];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                float c0, s0, c1, s1;
+                prologue_angle(t[u], rev[8 * j + e], c0, s0);
+                prologue_angle(t[u], rev[8 * j + e + 1], c1, s1);
+                const float u0 = a[e] * inv, w0 = b[e] * inv, u1 = a[e + 1] * inv, w1 = b[e + 1] * inv;
+                oa[e >> 1] = pack_bf16x2(u0 * c0 - w0 * s0, u1 * c1 - w1 * s1);
+                ob[e >> 1] = pack_bf16x2(u0 * s0 + w0 * c0, u1 * s1 + w1 * c1);
+            }
+            if (valid[u]) {
+                __nv_bfloat16* y = yb + ys.row(bh[u], p.H, t[u]) + 8 * j;
+                *reinterpret_cast<uint4*>(y) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+                *reinterpret_cast<uint4*>(y + H2) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+            }
         }
     }
 }
@@ -152,8 +193,8 @@ qk_prologue_bwd_kernel(const PrologueParams p) {
          row0 += (long long)gridDim.x * kRows) {    // warp-uniform bound, as in the forward kernel
         const long long row = row0 + (threadIdx.x & 31) / G;
         const bool valid = row < p.rows;
-        const int bh = valid ? (int)(row / p.T) : 0;
-        const int t = valid ? (int)(row - (long long)bh * p.T) : 0;
+        int bh = 0, t = 0;
+        if (valid) prologue_row(p, row, bh, t);
         const __nv_bfloat16* x = xb + xs.row(bh, p.H, t) + 8 * j;
         const __nv_bfloat16* g = gb + gs.row(bh, p.H, t) + 8 * j;
         float ga[8] = {}, gb2[8] = {}, xa[8] = {}, xb2[8] = {};
