@@ -28,16 +28,18 @@
 //   attn_dq_convert_kernel dQ = bf16(scale * fp32 accumulator).
 // dS is rounded to bf16 unscaled; the score scale is applied once per output
 // element, in the dK epilogue and in the dQ conversion.
-// The serial kernel below runs one query tile at a time through its five MMAs
-// and the P/dS warpgroup; it serves D = 128, whose accumulators fill all 512
-// TMEM columns (dQ reuses the S^T columns).
+// The kernel below serves D = 128, whose accumulators fill all 512 TMEM columns
+// (S^T, then P^T over it; dP^T, then dQ over it; dV; dK), so one query tile's
+// P/dS pass runs at a time.  Its five 8-step MMA chains go out from three
+// threads, each chain as soon as its operands and accumulator columns are free;
+// Q has a two-stage ring and dO one buffer (dO's last reader, dV, comes first).
 #pragma once
 
 #include "attn_fwd.cuh"
 
 namespace gpt_attn {
 
-constexpr int kBwdThreads = 320;     // 10 warps
+constexpr int kBwdThreads = 384;     // 12 warps
 
 struct BwdParams {
     const float* lse2;      // [BH, T_pad]  lse * log2(e); +inf past T
@@ -67,38 +69,42 @@ __device__ __forceinline__ int bwd_last_tile(const BwdParams& p, int bh, int kt,
 
 template <int D>
 struct BwdCfg {
-    static constexpr int kStages = (D == 64) ? 2 : 1;      // Q/dO ring depth (shared-memory bound)
+    static constexpr int kStages = 2;                       // Q/dO ring depth
     static constexpr int kTileBytes = kTile * D * 2;
     static constexpr uint32_t kColS = 0;                    // S^T, then P^T (bf16) over its first 64 columns
-    static constexpr uint32_t kColDP = 128;                 // dP^T
+    static constexpr uint32_t kColDP = 128;                 // dP^T, then dQ (D = 128)
     static constexpr uint32_t kColDV = 256;
     static constexpr uint32_t kColDK = 256 + D;
-    static constexpr uint32_t kColDQ = (D == 64) ? 384 : 0; // D = 128: dQ reuses the S^T columns
-    static constexpr bool kDqAliasesS = (D != 64);
+    static constexpr uint32_t kColDQ = (D == 64) ? 384 : kColDP;
 };
 
+// K and V of the unit, a two-stage ring of Q tiles (with their rows' lse, Delta and document
+// bounds), one dO tile and the dS^T tile: 195 KB for D = 128.  Q's last reader (dK) comes at the
+// end of a tile, dO's (dV) early, so Q gets the second stage.
 template <int D>
 struct BwdSmem {
     using C = BwdCfg<D>;
     alignas(1024) uint8_t k[C::kTileBytes];
     alignas(1024) uint8_t v[C::kTileBytes];
     alignas(1024) uint8_t q[C::kStages][C::kTileBytes];
-    alignas(1024) uint8_t dout[C::kStages][C::kTileBytes];
+    alignas(1024) uint8_t dout[C::kTileBytes];
     alignas(1024) uint8_t ds[kTile * kTile * 2];           // dS^T bf16 [key][query], two 64-query halves
     alignas(16) float lse2[C::kStages][kTile];
     alignas(16) float delta[C::kStages][kTile];
     alignas(16) int lower[C::kStages][kTile];               // document masks only
     uint64_t bar_kv;
-    uint64_t bar_qdo_full[C::kStages];
-    uint64_t bar_qdo_empty[C::kStages];
+    uint64_t bar_q_full[C::kStages];     // Q, lse, Delta (and bounds) of a query tile landed
+    uint64_t bar_q_empty[C::kStages];    // dK done with the stage (S finished long before)
+    uint64_t bar_do_full;
+    uint64_t bar_do_empty;               // dV done with dO (dP finished long before)
     uint64_t bar_s_full;
     uint64_t bar_dp_full;
     uint64_t bar_p_full;
     uint64_t bar_ds_full;
-    uint64_t bar_dv_done;
-    uint64_t bar_ds_empty;
+    uint64_t bar_dv_done;         // dV(g) finished reading P^T(g) out of the S^T columns
+    uint64_t bar_ds_empty;        // dK(g) and dQ(g) finished reading dS^T(g)
     uint64_t bar_dq_full;
-    uint64_t bar_dq_empty;
+    uint64_t bar_dq_empty;        // dQ(g) copied out of the dP^T columns
     uint64_t bar_dkdv_full;
     uint64_t bar_drain;
     uint32_t tmem_base;
@@ -217,19 +223,21 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     if (threadIdx.x == 0) {
         mbar_init(&sm.bar_kv, 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.bar_qdo_full[s], 1);
-            mbar_init(&sm.bar_qdo_empty[s], 1);
+            mbar_init(&sm.bar_q_full[s], 1);
+            mbar_init(&sm.bar_q_empty[s], 1);
         }
+        mbar_init(&sm.bar_do_full, 1);
+        mbar_init(&sm.bar_do_empty, 1);
         mbar_init(&sm.bar_s_full, 1);
         mbar_init(&sm.bar_dp_full, 1);
         mbar_init(&sm.bar_p_full, 128);
         mbar_init(&sm.bar_ds_full, 128);
         mbar_init(&sm.bar_dv_done, 1);
-        mbar_init(&sm.bar_ds_empty, 1);
+        mbar_init(&sm.bar_ds_empty, 2);             // dK issuer + dQ issuer
         mbar_init(&sm.bar_dq_full, 1);
         mbar_init(&sm.bar_dq_empty, 128);
         mbar_init(&sm.bar_dkdv_full, 1);
-        mbar_init(&sm.bar_drain, 1);
+        mbar_init(&sm.bar_drain, 3);                // the three MMA-issuing threads
         sm.abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -257,30 +265,43 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 tma_load_4d(sm.k + b * 16384, &tm_k, &sm.bar_kv, b * 64, k0, hh, bb);
                 tma_load_4d(sm.v + b * 16384, &tm_v, &sm.bar_kv, b * 64, k0, hh, bb);
             }
-            int it = 0;
-            for (; it < n_q; ++it) {
+            int nq = 0, ndo = 0;           // Q and dO tiles whose loads were issued
+            for (int it = 0; it < n_q; ++it) {
                 const int s = it % kStages;
                 const int n = it / kStages;
-                if (n > 0 && !mbar_wait(&sm.bar_qdo_empty[s], (n - 1) & 1, ac)) break;
+                if (n > 0 && !mbar_wait(&sm.bar_q_empty[s], (n - 1) & 1, ac)) break;
+                if (debug_skip_load(2, it)) continue;           // debug builds: exercise the abort path
                 const int q0 = (qt_lo + it) * kTile;
-                mbar_arrive_expect_tx(&sm.bar_qdo_full[s], 2 * kTileBytes + (p.lower2 ? 3 : 2) * kTile * 4);
-                for (int b = 0; b < kBoxes; ++b) {
-                    tma_load_4d(sm.q[s] + b * 16384, &tm_q, &sm.bar_qdo_full[s], b * 64, q0, hh, bb);
-                    tma_load_4d(sm.dout[s] + b * 16384, &tm_do, &sm.bar_qdo_full[s], b * 64, q0, hh, bb);
-                }
+                mbar_arrive_expect_tx(&sm.bar_q_full[s], kTileBytes + (p.lower2 ? 3 : 2) * kTile * 4);
+                for (int b = 0; b < kBoxes; ++b)
+                    tma_load_4d(sm.q[s] + b * 16384, &tm_q, &sm.bar_q_full[s], b * 64, q0, hh, bb);
                 const size_t roff = (size_t)bh * p.T_pad + q0;
-                bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
-                bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_qdo_full[s]);
-                if (p.lower2) bulk_load(sm.lower[s], p.lower2 + roff, kTile * 4, &sm.bar_qdo_full[s]);
+                bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_q_full[s]);
+                bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_q_full[s]);
+                if (p.lower2) bulk_load(sm.lower[s], p.lower2 + roff, kTile * 4, &sm.bar_q_full[s]);
+                nq = it + 1;
+                if (it > 0 && !mbar_wait(&sm.bar_do_empty, (it - 1) & 1, ac)) break;
+                mbar_arrive_expect_tx(&sm.bar_do_full, kTileBytes);
+                for (int b = 0; b < kBoxes; ++b)
+                    tma_load_4d(sm.dout + b * 16384, &tm_do, &sm.bar_do_full, b * 64, q0, hh, bb);
+                ndo = it + 1;
             }
             if (sm.abort_flag) {
+                // Let every load already issued land before the CTA exits.
                 mbar_wait_drain(&sm.bar_kv, 0, p.timeout_ns);
-                for (int r = (it > kStages ? it - kStages : 0); r < it; ++r)
-                    mbar_wait_drain(&sm.bar_qdo_full[r % kStages], (r / kStages) & 1, p.timeout_ns);
+                for (int r = (nq > kStages ? nq - kStages : 0); r < nq; ++r)
+                    mbar_wait_drain(&sm.bar_q_full[r % kStages], (r / kStages) & 1, p.timeout_ns);
+                if (ndo > 0) mbar_wait_drain(&sm.bar_do_full, (ndo - 1) & 1, p.timeout_ns);
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ MMA issuers
+        // One thread issues one tcgen05.mma per ~130 cycles, so the five 8-step chains of a tile
+        // go out from three threads, each as soon as its operands and accumulator are free:
+        //   warp 1: S^T(g) once dV(g-1) has read P^T(g-1) out of the S^T columns
+        //   warp 2: dP^T(g) once dQ(g-1) has been copied out of the dP^T columns, then dQ(g) into
+        //           those columns once the P/dS warpgroup has read dP^T(g) and written dS^T(g)
+        //   warp 3: dV(g) once P^T(g) is in TMEM, then dK(g) once dS^T(g) is in shared memory
         if (lane == 0) {
             const uint32_t k_addr = smem_u32(sm.k);
             const uint32_t v_addr = smem_u32(sm.v);
@@ -290,66 +311,69 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const int s = it % kStages;
                 const uint32_t ph = (it / kStages) & 1;
                 const uint32_t q_addr = smem_u32(sm.q[s]);
-                const uint32_t do_addr = smem_u32(sm.dout[s]);
-                if (!mbar_wait(&sm.bar_qdo_full[s], ph, ac)) break;
-                if (it > 0) {
-                    // S^T columns: the previous dV MMA read P^T from them (and, for D = 128, the
-                    // previous dQ was accumulated there and must have been read out).
-                    if (!mbar_wait(&sm.bar_dv_done, (it - 1) & 1, ac)) break;
-                    if (C::kDqAliasesS && !mbar_wait(&sm.bar_dq_empty, (it - 1) & 1, ac)) break;
+                const uint32_t do_addr = smem_u32(sm.dout);
+                if (warp == 1) {
+                    if (!(ok = mbar_wait(&sm.bar_q_full[s], ph, ac))) break;
+                    if (it > 0 && !(ok = mbar_wait(&sm.bar_dv_done, (it - 1) & 1, ac))) break;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_ss(tmem + C::kColS, sw128_desc(k_addr + off, 16, 1024),
+                               sw128_desc(q_addr + off, 16, 1024), kIdescSS, kk > 0);
+                    }
+                    mma_commit(&sm.bar_s_full);
+                } else if (warp == 2) {
+                    if (!(ok = mbar_wait(&sm.bar_do_full, it & 1, ac))) break;
+                    if (it > 0 && !(ok = mbar_wait(&sm.bar_dq_empty, (it - 1) & 1, ac))) break;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_ss(tmem + C::kColDP, sw128_desc(v_addr + off, 16, 1024),
+                               sw128_desc(do_addr + off, 16, 1024), kIdescSS, kk > 0);
+                    }
+                    mma_commit(&sm.bar_dp_full);
+                    // dQ = dS K
+                    if (!(ok = mbar_wait(&sm.bar_ds_full, it & 1, ac))) break;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
+                               sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
+                    mma_commit(&sm.bar_dq_full);
+                    mma_commit(&sm.bar_ds_empty);
+                } else {
+                    // dV += P^T dO
+                    if (!(ok = mbar_wait(&sm.bar_p_full, it & 1, ac))) break;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int kk = 0; kk < kTile / 16; ++kk)
+                        mma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8,
+                               sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdescKxMN,
+                               (it > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&sm.bar_dv_done);
+                    mma_commit(&sm.bar_do_empty);          // dV was dO's last reader
+                    // dK += dS^T Q
+                    if (!(ok = mbar_wait(&sm.bar_ds_full, it & 1, ac))) break;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int kk = 0; kk < kTile / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
+                               sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN,
+                               (it > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&sm.bar_ds_empty);
+                    mma_commit(&sm.bar_q_empty[s]);        // dK was Q's last reader
                 }
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_ss(tmem + C::kColS, sw128_desc(k_addr + off, 16, 1024), sw128_desc(q_addr + off, 16, 1024),
-                           kIdescSS, kk > 0);
-                }
-                mma_commit(&sm.bar_s_full);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_ss(tmem + C::kColDP, sw128_desc(v_addr + off, 16, 1024),
-                           sw128_desc(do_addr + off, 16, 1024), kIdescSS, kk > 0);
-                }
-                mma_commit(&sm.bar_dp_full);
-                // dV += P^T dO
-                if (!mbar_wait(&sm.bar_p_full, it & 1, ac)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8, sw128_desc(do_addr + kk * 2048, 16384, 1024),
-                           kIdescKxMN, (it > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&sm.bar_dv_done);
-                // dK += dS^T Q
-                if (!mbar_wait(&sm.bar_ds_full, it & 1, ac)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
-                           sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN, (it > 0 || kk > 0) ? 1u : 0u);
-                }
-                // dQ = dS K (needs the dQ columns free; for D = 128 also the dV MMA done with P^T)
-                if (C::kDqAliasesS) {
-                    if (!mbar_wait(&sm.bar_dv_done, it & 1, ac)) break;
-                } else if (it > 0) {
-                    if (!mbar_wait(&sm.bar_dq_empty, (it - 1) & 1, ac)) break;
-                }
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
-                           sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
-                mma_commit(&sm.bar_dq_full);
-                mma_commit(&sm.bar_qdo_empty[s]);
-                mma_commit(&sm.bar_ds_empty);
             }
-            mma_commit(&sm.bar_dkdv_full);
+            if (warp == 3 && ok) mma_commit(&sm.bar_dkdv_full);
+            // No MMA of this thread may still be running when TMEM is released.
             mma_commit(&sm.bar_drain);
             mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
         }
-    } else if (warp < 6) {
+    } else if (warp < 8) {
         // ------------------------------------------------------------ P / dS warpgroup (thread = key row)
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
@@ -361,13 +385,11 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         bool ok = true;
         for (int it = 0; it < n_q; ++it) {
             const int s = it % kStages;
-            const uint32_t ph = (it / kStages) & 1;
             const int qt = qt_lo + it;
             const int q0 = qt * kTile;
-            if (!warp_wait(&sm.bar_qdo_full[s], ph, ac)) { ok = false; break; }
+            if (!warp_wait(&sm.bar_q_full[s], (it / kStages) & 1, ac)) { ok = false; break; }
             if (!warp_wait(&sm.bar_s_full, it & 1, ac)) { ok = false; break; }
             if (!warp_wait(&sm.bar_dp_full, it & 1, ac)) { ok = false; break; }
-            if (it > 0 && !warp_wait(&sm.bar_ds_empty, (it - 1) & 1, ac)) { ok = false; break; }
             tc_fence_after();
             // The tile needs the per-element mask if it holds the diagonal or some query of it
             // starts seeing keys after this key tile's first key (lower bounds do not decrease
@@ -413,6 +435,12 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     dk[e >> 1] = pack_bf16x2(d0, d1);
                 }
                 tmem_st16(t_lane + C::kColS + c * 16, pk);
+                // dS^T(it) may go into the shared buffer once dK(it-1) and dQ(it-1) have read it.
+                if (c == 0 && it > 0 && !warp_wait(&sm.bar_ds_empty, (it - 1) & 1, ac)) {
+                    tmem_wait_st();                    // no store may be left in flight
+                    ok = false;
+                    break;
+                }
                 // dS^T row r, queries [32c, 32c + 32): 4 chunks of 16 bytes in half c/2, swizzled by row.
                 const uint32_t half = ds_row + (c >> 1) * 16384;
 #pragma unroll
@@ -421,6 +449,7 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     st_shared_v4(half + chunk * 16, dk[4 * t], dk[4 * t + 1], dk[4 * t + 2], dk[4 * t + 3]);
                 }
             }
+            if (!ok) break;
             tmem_wait_st();
             tc_fence_before();
             fence_proxy_async_smem();
