@@ -39,7 +39,7 @@
 
 namespace gpt_attn {
 
-constexpr int kBwdThreads = 384;     // 12 warps
+constexpr int kBwdThreads = 512;     // 16 warps
 
 struct BwdParams {
     const float* lse2;      // [BH, T_pad]  lse * log2(e); +inf past T
@@ -230,8 +230,8 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         mbar_init(&sm.bar_do_empty, 1);
         mbar_init(&sm.bar_s_full, 1);
         mbar_init(&sm.bar_dp_full, 1);
-        mbar_init(&sm.bar_p_full, 128);
-        mbar_init(&sm.bar_ds_full, 128);
+        mbar_init(&sm.bar_p_full, 256);             // both P/dS warpgroups
+        mbar_init(&sm.bar_ds_full, 256);
         mbar_init(&sm.bar_dv_done, 1);
         mbar_init(&sm.bar_ds_empty, 2);             // dK issuer + dQ issuer
         mbar_init(&sm.bar_dq_full, 1);
@@ -349,7 +349,7 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     tc_fence_after();
 #pragma unroll 1
                     for (int kk = 0; kk < kTile / 16; ++kk)
-                        mma_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8,
+                        mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
                                sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdescKxMN,
                                (it > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(&sm.bar_dv_done);
@@ -373,8 +373,12 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             mma_commit(&sm.bar_drain);
             mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
         }
-    } else if (warp < 8) {
-        // ------------------------------------------------------------ P / dS warpgroup (thread = key row)
+    } else if (warp < 12) {
+        // ------------------------------------------------------------ P / dS warpgroups (thread = key row)
+        // Warpgroup h takes query columns [64h, 64h + 64) of each tile and writes their P^T over
+        // S^T columns it has read itself: queries 64h + q go to bf16 column 64h + q/2 of the S^T
+        // block, so neither warpgroup overwrites scores the other still has to read.
+        const int h = (warp - 4) >> 2;
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
         const int key = k0 + r;
@@ -399,7 +403,7 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             const float2* lse2 = reinterpret_cast<const float2*>(sm.lse2[s]);
             const float2* dlt = reinterpret_cast<const float2*>(sm.delta[s]);
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * h; c < 2 * h + 2; ++c) {
                 uint32_t rs[32], rd[32];
                 tmem_ld32(t_lane + C::kColS + c * 32, rs);
                 tmem_ld32(t_lane + C::kColDP + c * 32, rd);
@@ -434,9 +438,9 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     pk[e >> 1] = pack_bf16x2(p0, p1);
                     dk[e >> 1] = pack_bf16x2(d0, d1);
                 }
-                tmem_st16(t_lane + C::kColS + c * 16, pk);
+                tmem_st16(t_lane + C::kColS + h * 64 + (c & 1) * 16, pk);
                 // dS^T(it) may go into the shared buffer once dK(it-1) and dQ(it-1) have read it.
-                if (c == 0 && it > 0 && !warp_wait(&sm.bar_ds_empty, (it - 1) & 1, ac)) {
+                if (c == 2 * h && it > 0 && !warp_wait(&sm.bar_ds_empty, (it - 1) & 1, ac)) {
                     tmem_wait_st();                    // no store may be left in flight
                     ok = false;
                     break;
@@ -467,7 +471,7 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const uint32_t col0 = which == 0 ? C::kColDV : C::kColDK;
                 const float mul = which == 0 ? 1.f : p.scale;     // dK = scale * dS^T Q
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = h * D / 64; c < (h + 1) * D / 64; ++c) {     // this warpgroup's half of D
                     uint32_t rr[32];
                     tmem_ld32(t_lane + col0 + c * 32, rr);
                     tmem_wait_ld();
