@@ -252,127 +252,133 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const uint32_t tmem = sm.tmem_base;
     const AbortCtl ac{&sm.abort_flag, p.timeout_ns};
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-            tma_prefetch_desc(&tm_do);
-            const int hh = bh % p.H, bb = bh / p.H;
-            mbar_arrive_expect_tx(&sm.bar_kv, 2 * kTileBytes);
-            for (int b = 0; b < kBoxes; ++b) {
-                tma_load_4d(sm.k + b * 16384, &tm_k, &sm.bar_kv, b * 64, k0, hh, bb);
-                tma_load_4d(sm.v + b * 16384, &tm_v, &sm.bar_kv, b * 64, k0, hh, bb);
-            }
-            int nq = 0, ndo = 0;           // Q and dO tiles whose loads were issued
-            for (int it = 0; it < n_q; ++it) {
-                const int s = it % kStages;
-                const int n = it / kStages;
-                if (n > 0 && !mbar_wait(&sm.bar_q_empty[s], (n - 1) & 1, ac)) break;
-                if (debug_skip_load(2, it)) continue;           // debug builds: exercise the abort path
-                const int q0 = (qt_lo + it) * kTile;
-                mbar_arrive_expect_tx(&sm.bar_q_full[s], kTileBytes + (p.lower2 ? 3 : 2) * kTile * 4);
-                for (int b = 0; b < kBoxes; ++b)
-                    tma_load_4d(sm.q[s] + b * 16384, &tm_q, &sm.bar_q_full[s], b * 64, q0, hh, bb);
-                const size_t roff = (size_t)bh * p.T_pad + q0;
-                bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_q_full[s]);
-                bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_q_full[s]);
-                if (p.lower2) bulk_load(sm.lower[s], p.lower2 + roff, kTile * 4, &sm.bar_q_full[s]);
-                nq = it + 1;
-                if (it > 0 && !mbar_wait(&sm.bar_do_empty, (it - 1) & 1, ac)) break;
-                mbar_arrive_expect_tx(&sm.bar_do_full, kTileBytes);
-                for (int b = 0; b < kBoxes; ++b)
-                    tma_load_4d(sm.dout + b * 16384, &tm_do, &sm.bar_do_full, b * 64, q0, hh, bb);
-                ndo = it + 1;
-            }
-            if (sm.abort_flag) {
-                // Let every load already issued land before the CTA exits.
-                mbar_wait_drain(&sm.bar_kv, 0, p.timeout_ns);
-                for (int r = (nq > kStages ? nq - kStages : 0); r < nq; ++r)
-                    mbar_wait_drain(&sm.bar_q_full[r % kStages], (r / kStages) & 1, p.timeout_ns);
-                if (ndo > 0) mbar_wait_drain(&sm.bar_do_full, (ndo - 1) & 1, p.timeout_ns);
-            }
-        }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ MMA issuers
-        // One thread issues one tcgen05.mma per ~130 cycles, so the five 8-step chains of a tile
-        // go out from three threads, each as soon as its operands and accumulator are free:
-        //   warp 1: S^T(g) once dV(g-1) has read P^T(g-1) out of the S^T columns
-        //   warp 2: dP^T(g) once dQ(g-1) has been copied out of the dP^T columns, then dQ(g) into
-        //           those columns once the P/dS warpgroup has read dP^T(g) and written dS^T(g)
-        //   warp 3: dV(g) once P^T(g) is in TMEM, then dK(g) once dS^T(g) is in shared memory
-        if (lane == 0) {
-            const uint32_t k_addr = smem_u32(sm.k);
-            const uint32_t v_addr = smem_u32(sm.v);
-            const uint32_t ds_addr = smem_u32(sm.ds);
-            bool ok = mbar_wait(&sm.bar_kv, 0, ac);
-            for (int it = 0; ok && it < n_q; ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
-                const uint32_t q_addr = smem_u32(sm.q[s]);
-                const uint32_t do_addr = smem_u32(sm.dout);
-                if (warp == 1) {
-                    if (!(ok = mbar_wait(&sm.bar_q_full[s], ph, ac))) break;
-                    if (it > 0 && !(ok = mbar_wait(&sm.bar_dv_done, (it - 1) & 1, ac))) break;
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        mma_ss(tmem + C::kColS, sw128_desc(k_addr + off, 16, 1024),
-                               sw128_desc(q_addr + off, 16, 1024), kIdescSS, kk > 0);
-                    }
-                    mma_commit(&sm.bar_s_full);
-                } else if (warp == 2) {
-                    if (!(ok = mbar_wait(&sm.bar_do_full, it & 1, ac))) break;
-                    if (it > 0 && !(ok = mbar_wait(&sm.bar_dq_empty, (it - 1) & 1, ac))) break;
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        mma_ss(tmem + C::kColDP, sw128_desc(v_addr + off, 16, 1024),
-                               sw128_desc(do_addr + off, 16, 1024), kIdescSS, kk > 0);
-                    }
-                    mma_commit(&sm.bar_dp_full);
-                    // dQ = dS K
-                    if (!(ok = mbar_wait(&sm.bar_ds_full, it & 1, ac))) break;
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int kk = 0; kk < kTile / 16; ++kk)
-                        mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
-                               sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
-                    mma_commit(&sm.bar_dq_full);
-                    mma_commit(&sm.bar_ds_empty);
-                } else {
-                    // dV += P^T dO
-                    if (!(ok = mbar_wait(&sm.bar_p_full, it & 1, ac))) break;
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int kk = 0; kk < kTile / 16; ++kk)
-                        mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
-                               sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdescKxMN,
-                               (it > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(&sm.bar_dv_done);
-                    mma_commit(&sm.bar_do_empty);          // dV was dO's last reader
-                    // dK += dS^T Q
-                    if (!(ok = mbar_wait(&sm.bar_ds_full, it & 1, ac))) break;
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
-                               sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN,
-                               (it > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(&sm.bar_ds_empty);
-                    mma_commit(&sm.bar_q_empty[s]);        // dK was Q's last reader
+    // Launched with 128 registers per thread (512 x 128 = 65536): warpgroup 0 (producer and MMA
+    // issuers) drops to 56, the dQ writer takes 200 to hold a whole row of dQ, the P/dS warpgroups
+    // keep 128: 128 x (56 + 128 + 128 + 200) = 65536.
+    if (warp < 4) {
+        regs_dec<56>();
+        if (warp == 0) {
+            // ------------------------------------------------------------ producer
+            if (lane == 0) {
+                tma_prefetch_desc(&tm_q);
+                tma_prefetch_desc(&tm_k);
+                tma_prefetch_desc(&tm_v);
+                tma_prefetch_desc(&tm_do);
+                const int hh = bh % p.H, bb = bh / p.H;
+                mbar_arrive_expect_tx(&sm.bar_kv, 2 * kTileBytes);
+                for (int b = 0; b < kBoxes; ++b) {
+                    tma_load_4d(sm.k + b * 16384, &tm_k, &sm.bar_kv, b * 64, k0, hh, bb);
+                    tma_load_4d(sm.v + b * 16384, &tm_v, &sm.bar_kv, b * 64, k0, hh, bb);
+                }
+                int nq = 0, ndo = 0;           // Q and dO tiles whose loads were issued
+                for (int it = 0; it < n_q; ++it) {
+                    const int s = it % kStages;
+                    const int n = it / kStages;
+                    if (n > 0 && !mbar_wait(&sm.bar_q_empty[s], (n - 1) & 1, ac)) break;
+                    if (debug_skip_load(2, it)) continue;           // debug builds: exercise the abort path
+                    const int q0 = (qt_lo + it) * kTile;
+                    mbar_arrive_expect_tx(&sm.bar_q_full[s], kTileBytes + (p.lower2 ? 3 : 2) * kTile * 4);
+                    for (int b = 0; b < kBoxes; ++b)
+                        tma_load_4d(sm.q[s] + b * 16384, &tm_q, &sm.bar_q_full[s], b * 64, q0, hh, bb);
+                    const size_t roff = (size_t)bh * p.T_pad + q0;
+                    bulk_load(sm.lse2[s], p.lse2 + roff, kTile * 4, &sm.bar_q_full[s]);
+                    bulk_load(sm.delta[s], p.delta + roff, kTile * 4, &sm.bar_q_full[s]);
+                    if (p.lower2) bulk_load(sm.lower[s], p.lower2 + roff, kTile * 4, &sm.bar_q_full[s]);
+                    nq = it + 1;
+                    if (it > 0 && !mbar_wait(&sm.bar_do_empty, (it - 1) & 1, ac)) break;
+                    mbar_arrive_expect_tx(&sm.bar_do_full, kTileBytes);
+                    for (int b = 0; b < kBoxes; ++b)
+                        tma_load_4d(sm.dout + b * 16384, &tm_do, &sm.bar_do_full, b * 64, q0, hh, bb);
+                    ndo = it + 1;
+                }
+                if (sm.abort_flag) {
+                    // Let every load already issued land before the CTA exits.
+                    mbar_wait_drain(&sm.bar_kv, 0, p.timeout_ns);
+                    for (int r = (nq > kStages ? nq - kStages : 0); r < nq; ++r)
+                        mbar_wait_drain(&sm.bar_q_full[r % kStages], (r / kStages) & 1, p.timeout_ns);
+                    if (ndo > 0) mbar_wait_drain(&sm.bar_do_full, (ndo - 1) & 1, p.timeout_ns);
                 }
             }
-            if (warp == 3 && ok) mma_commit(&sm.bar_dkdv_full);
-            // No MMA of this thread may still be running when TMEM is released.
-            mma_commit(&sm.bar_drain);
-            mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
-        }
+        } else {
+            // ------------------------------------------------------------ MMA issuers
+            // One thread issues one tcgen05.mma per ~130 cycles, so the five 8-step chains of a tile
+            // go out from three threads, each as soon as its operands and accumulator are free:
+            //   warp 1: S^T(g) once dV(g-1) has read P^T(g-1) out of the S^T columns
+            //   warp 2: dP^T(g) once dQ(g-1) has been copied out of the dP^T columns, then dQ(g) into
+            //           those columns once the P/dS warpgroup has read dP^T(g) and written dS^T(g)
+            //   warp 3: dV(g) once P^T(g) is in TMEM, then dK(g) once dS^T(g) is in shared memory
+            if (lane == 0) {
+                const uint32_t k_addr = smem_u32(sm.k);
+                const uint32_t v_addr = smem_u32(sm.v);
+                const uint32_t ds_addr = smem_u32(sm.ds);
+                bool ok = mbar_wait(&sm.bar_kv, 0, ac);
+                for (int it = 0; ok && it < n_q; ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1;
+                    const uint32_t q_addr = smem_u32(sm.q[s]);
+                    const uint32_t do_addr = smem_u32(sm.dout);
+                    if (warp == 1) {
+                        if (!(ok = mbar_wait(&sm.bar_q_full[s], ph, ac))) break;
+                        if (it > 0 && !(ok = mbar_wait(&sm.bar_dv_done, (it - 1) & 1, ac))) break;
+                        tc_fence_after();
+    #pragma unroll 1
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                            mma_ss(tmem + C::kColS, sw128_desc(k_addr + off, 16, 1024),
+                                   sw128_desc(q_addr + off, 16, 1024), kIdescSS, kk > 0);
+                        }
+                        mma_commit(&sm.bar_s_full);
+                    } else if (warp == 2) {
+                        if (!(ok = mbar_wait(&sm.bar_do_full, it & 1, ac))) break;
+                        if (it > 0 && !(ok = mbar_wait(&sm.bar_dq_empty, (it - 1) & 1, ac))) break;
+                        tc_fence_after();
+    #pragma unroll 1
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                            mma_ss(tmem + C::kColDP, sw128_desc(v_addr + off, 16, 1024),
+                                   sw128_desc(do_addr + off, 16, 1024), kIdescSS, kk > 0);
+                        }
+                        mma_commit(&sm.bar_dp_full);
+                        // dQ = dS K
+                        if (!(ok = mbar_wait(&sm.bar_ds_full, it & 1, ac))) break;
+                        tc_fence_after();
+    #pragma unroll 1
+                        for (int kk = 0; kk < kTile / 16; ++kk)
+                            mma_ss(tmem + C::kColDQ, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
+                                   sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdescMNxMN, kk > 0);
+                        mma_commit(&sm.bar_dq_full);
+                        mma_commit(&sm.bar_ds_empty);
+                    } else {
+                        // dV += P^T dO
+                        if (!(ok = mbar_wait(&sm.bar_p_full, it & 1, ac))) break;
+                        tc_fence_after();
+    #pragma unroll 1
+                        for (int kk = 0; kk < kTile / 16; ++kk)
+                            mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
+                                   sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdescKxMN,
+                                   (it > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(&sm.bar_dv_done);
+                        mma_commit(&sm.bar_do_empty);          // dV was dO's last reader
+                        // dK += dS^T Q
+                        if (!(ok = mbar_wait(&sm.bar_ds_full, it & 1, ac))) break;
+                        tc_fence_after();
+    #pragma unroll 1
+                        for (int kk = 0; kk < kTile / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                            mma_ss(tmem + C::kColDK, sw128_desc(ds_addr + off, 16, 1024),
+                                   sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdescKxMN,
+                                   (it > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(&sm.bar_ds_empty);
+                        mma_commit(&sm.bar_q_empty[s]);        // dK was Q's last reader
+                    }
+                }
+                if (warp == 3 && ok) mma_commit(&sm.bar_dkdv_full);
+                // No MMA of this thread may still be running when TMEM is released.
+                mma_commit(&sm.bar_drain);
+                mbar_wait_drain(&sm.bar_drain, 0, p.timeout_ns);
+            }
+    }
     } else if (warp < 12) {
         // ------------------------------------------------------------ P / dS warpgroups (thread = key row)
         // Warpgroup h takes query columns [64h, 64h + 64) of each tile and writes their P^T over
@@ -489,6 +495,7 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             }
         }
     } else {
+        regs_inc<200>();
         // ------------------------------------------------------------ dQ writer warpgroup (thread = query row)
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
@@ -498,20 +505,29 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             if (!warp_wait(&sm.bar_dq_full, it & 1, ac)) break;
             tc_fence_after();
             float* dst = p.dq_acc + ((size_t)bh * p.T + (q < p.T ? q : 0)) * D;
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t rr[32];
-                tmem_ld32(t_lane + C::kColDQ + c * 32, rr);
-                tmem_wait_ld();
-                if (q < p.T) {
-#pragma unroll
-                    for (int v4 = 0; v4 < 8; ++v4)
-                        red_add_v4(dst + c * 32 + 4 * v4, __uint_as_float(rr[4 * v4]), __uint_as_float(rr[4 * v4 + 1]),
-                                   __uint_as_float(rr[4 * v4 + 2]), __uint_as_float(rr[4 * v4 + 3]));
-                }
-            }
+            // The whole row comes out of TMEM first, so the next tile's dP^T may overwrite the
+            // columns before the adds below are issued.
+            static_assert(D == 128, "the dQ writer holds a row as four 32-column pieces");
+            uint32_t r0[32], r1[32], r2[32], r3[32];
+            tmem_ld32(t_lane + C::kColDQ, r0);
+            tmem_ld32(t_lane + C::kColDQ + 32, r1);
+            tmem_ld32(t_lane + C::kColDQ + 64, r2);
+            tmem_ld32(t_lane + C::kColDQ + 96, r3);
+            tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.bar_dq_empty);
+            if (q < p.T) {
+                auto add32 = [&](float* d, const uint32_t (&v)[32]) {
+#pragma unroll
+                    for (int v4 = 0; v4 < 8; ++v4)
+                        red_add_v4(d + 4 * v4, __uint_as_float(v[4 * v4]), __uint_as_float(v[4 * v4 + 1]),
+                                   __uint_as_float(v[4 * v4 + 2]), __uint_as_float(v[4 * v4 + 3]));
+                };
+                add32(dst, r0);
+                add32(dst + 32, r1);
+                add32(dst + 64, r2);
+                add32(dst + 96, r3);
+            }
         }
     }
 
