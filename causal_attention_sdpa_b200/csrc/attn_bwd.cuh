@@ -22,9 +22,9 @@
 //                            dV  += P^T dO         (P^T read from TMEM)
 //                            dK  += dS^T Q         (dS^T from shared memory)
 //                            dQ   = dS K           (same shared tile, MN-major)
-//                          dQ is added into the fp32 accumulator by TMA bulk
-//                          reduce-adds (D=64) or vector red.global.add (D=128)
-//                          from a dedicated warpgroup.
+//                          dQ is staged in shared memory and added into the
+//                          fp32 accumulator by TMA bulk reduce-adds from a
+//                          dedicated warpgroup.
 //   attn_dq_convert_kernel dQ = bf16(scale * fp32 accumulator).
 // dS is rounded to bf16 unscaled; the score scale is applied once per output
 // element, in the dK epilogue and in the dQ conversion.
@@ -89,6 +89,8 @@ struct BwdSmem {
     alignas(1024) uint8_t q[C::kStages][C::kTileBytes];
     alignas(1024) uint8_t dout[C::kTileBytes];
     alignas(1024) uint8_t ds[kTile * kTile * 2];           // dS^T bf16 [key][query], two 64-query halves
+    // 32 columns of dQ in fp32 for one bulk reduce-add into the accumulator, 128B-swizzled
+    alignas(1024) uint8_t stage[kTile * 32 * 4];
     alignas(16) float lse2[C::kStages][kTile];
     alignas(16) float delta[C::kStages][kTile];
     alignas(16) int lower[C::kStages][kTile];               // document masks only
@@ -105,6 +107,8 @@ struct BwdSmem {
     uint64_t bar_ds_empty;        // dK(g) and dQ(g) finished reading dS^T(g)
     uint64_t bar_dq_full;
     uint64_t bar_dq_empty;        // dQ(g) copied out of the dP^T columns
+    uint64_t bar_stage_full;      // the dQ writer has staged a 32-column piece
+    uint64_t bar_stage_free;      // the piece's reduce-add has read the staging buffer
     uint64_t bar_dkdv_full;
     uint64_t bar_drain;
     uint32_t tmem_base;
@@ -194,7 +198,7 @@ attn_dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict_
 template <int D, typename Mask>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_dq,
                 const BwdParams p, const __grid_constant__ Mask mask) {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -236,6 +240,8 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         mbar_init(&sm.bar_ds_empty, 2);             // dK issuer + dQ issuer
         mbar_init(&sm.bar_dq_full, 1);
         mbar_init(&sm.bar_dq_empty, 128);
+        mbar_init(&sm.bar_stage_full, 128);
+        mbar_init(&sm.bar_stage_free, 1);
         mbar_init(&sm.bar_dkdv_full, 1);
         mbar_init(&sm.bar_drain, 3);                // the three MMA-issuing threads
         sm.abort_flag = 0;
@@ -253,10 +259,10 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const AbortCtl ac{&sm.abort_flag, p.timeout_ns};
 
     // Launched with 128 registers per thread (512 x 128 = 65536): warpgroup 0 (producer and MMA
-    // issuers) drops to 56, the dQ writer takes 200 to hold a whole row of dQ, the P/dS warpgroups
-    // keep 128: 128 x (56 + 128 + 128 + 200) = 65536.
+    // issuers) drops to 64, the P/dS warpgroups take 136, the dQ writer 176 to hold a whole row of
+    // dQ: 128 x (64 + 136 + 136 + 176) = 65536.
     if (warp < 4) {
-        regs_dec<56>();
+        regs_dec<64>();
         if (warp == 0) {
             // ------------------------------------------------------------ producer
             if (lane == 0) {
@@ -380,6 +386,7 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             }
     }
     } else if (warp < 12) {
+        regs_inc<136>();
         // ------------------------------------------------------------ P / dS warpgroups (thread = key row)
         // Warpgroup h takes query columns [64h, 64h + 64) of each tile and writes their P^T over
         // S^T columns it has read itself: queries 64h + q go to bf16 column 64h + q/2 of the S^T
@@ -495,18 +502,19 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             }
         }
     } else {
-        regs_inc<200>();
+        regs_inc<176>();
         // ------------------------------------------------------------ dQ writer warpgroup (thread = query row)
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
         for (int it = 0; it < n_q; ++it) {
-            const int q = (qt_lo + it) * kTile + r;
             if (!warp_wait(&sm.bar_dq_full, it & 1, ac)) break;
             tc_fence_after();
-            float* dst = p.dq_acc + ((size_t)bh * p.T + (q < p.T ? q : 0)) * D;
             // The whole row comes out of TMEM first, so the next tile's dP^T may overwrite the
-            // columns before the adds below are issued.
+            // columns at once.  Then it is added into the fp32 accumulator in four 32-column
+            // pieces, each staged in shared memory and sent by one TMA bulk reduce-add (rows past T
+            // are skipped): the tensor cores' shared-memory reads slow down badly under as many
+            // vector red.global.add from the LSU.
             static_assert(D == 128, "the dQ writer holds a row as four 32-column pieces");
             uint32_t r0[32], r1[32], r2[32], r3[32];
             tmem_ld32(t_lane + C::kColDQ, r0);
@@ -516,19 +524,30 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.bar_dq_empty);
-            if (q < p.T) {
-                auto add32 = [&](float* d, const uint32_t (&v)[32]) {
+            const uint32_t row_a = smem_u32(sm.stage) + r * 128;
+            auto put = [&](int j, const uint32_t (&v)[32]) -> bool {
+                const int n = it * 4 + j;                 // pieces staged so far
+                if (n > 0 && !warp_wait(&sm.bar_stage_free, (n - 1) & 1, ac)) return false;
 #pragma unroll
-                    for (int v4 = 0; v4 < 8; ++v4)
-                        red_add_v4(d + 4 * v4, __uint_as_float(v[4 * v4]), __uint_as_float(v[4 * v4 + 1]),
-                                   __uint_as_float(v[4 * v4 + 2]), __uint_as_float(v[4 * v4 + 3]));
-                };
-                add32(dst, r0);
-                add32(dst + 32, r1);
-                add32(dst + 64, r2);
-                add32(dst + 96, r3);
-            }
+                for (int c = 0; c < 8; ++c)
+                    st_shared_v4(row_a + ((c ^ (r & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.bar_stage_full);
+                bool lok = true;
+                if (warp == 12 && lane == 0) {
+                    lok = mbar_wait(&sm.bar_stage_full, n & 1, ac);
+                    if (lok) {
+                        tma_reduce_add_3d(&tm_dq, sm.stage, j * 32, (qt_lo + it) * kTile, bh);
+                        bulk_commit_group();
+                        bulk_wait_group_read0();
+                        mbar_arrive(&sm.bar_stage_free);
+                    }
+                }
+                return __all_sync(0xffffffffu, lok);
+            };
+            if (!put(0, r0) || !put(1, r1) || !put(2, r2) || !put(3, r3)) break;
         }
+        if (warp == 12 && lane == 0) bulk_wait_group0();   // every reduce-add has landed
     }
 
     tc_fence_before();

@@ -321,14 +321,16 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
             attn_bwd_kernel<MaskParams><<<pgrid, kBwd64Threads, smem, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p, mask);
         }
     } else {
+        CUtensorMap mdq;
+        if (!make_tmap_f32_acc(&mdq, w.dq_acc, BH, T, D)) return GPT_ATTN_ERR_CUDA;
         const size_t smem = sizeof(BwdSmem<D>) + 1024;
         if (plain_window(mask)) {
             if (!set_smem(attn_bwd_serial_kernel<D, WindowMask>, smem)) return GPT_ATTN_ERR_CUDA;
-            attn_bwd_serial_kernel<D, WindowMask><<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p,
+            attn_bwd_serial_kernel<D, WindowMask><<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdq, p,
                                                                                  WindowMask{mask.window});
         } else {
             if (!set_smem(attn_bwd_serial_kernel<D, MaskParams>, smem)) return GPT_ATTN_ERR_CUDA;
-            attn_bwd_serial_kernel<D, MaskParams><<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p, mask);
+            attn_bwd_serial_kernel<D, MaskParams><<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdq, p, mask);
         }
     }
     return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
