@@ -440,8 +440,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!ok || u < 0) break;
             const Bwd64Unit w = bwd64_unit(u, p, mask);
             const int kb = n & 1;
-            // dK / dV of this unit (thread = key row): copied out of TMEM as soon as the unit's last
-            // dQ is complete, before that dQ is reduced, so the next unit's first dV/dK can start.
+            // dK / dV of this unit (thread = key row): copied out of TMEM once the unit's last dQ
+            // has been copied out and staged for its reduce-add.
             // They are staged as bf16 128B-swizzled tiles in this unit's V and K buffers, which no
             // MMA reads any more (the last dP and dQ of the unit completed before dkdv_full), and
             // written with TMA tile stores (rows past T are clipped), so every warp writes whole
@@ -489,7 +489,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int b = g & 1;
                 if (!warp_wait(&sm.bar_dq_full, g & 1, ac)) { ok = false; break; }
                 tc_fence_after();
-                if (i == w.n_q - 1 && !(ok = __all_sync(0xffffffffu, write_dkdv()))) break;
                 uint32_t rr[64];
                 tmem_ld32(t_lane + C::kColDQ, *reinterpret_cast<uint32_t(*)[32]>(&rr[0]));
                 tmem_ld32(t_lane + C::kColDQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&rr[32]));
@@ -518,6 +517,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     bulk_wait_group_read0();
                     mbar_arrive(&sm.bar_ds_empty[b]);        // dS(g + 2) may be written now
                 }
+                // The unit's dK and dV go out after its last dQ has been handed on, so the next
+                // tile's dQ and dS buffer are not held up behind their copy and stores.
+                if (i == w.n_q - 1 && !(ok = __all_sync(0xffffffffu, write_dkdv()))) break;
             }
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
