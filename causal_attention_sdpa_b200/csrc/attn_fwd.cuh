@@ -279,7 +279,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // tensor pipe busy with 128-row MMAs of N <= 128, several streams can.
         //   warp 1: S0 = Q0 K_j^T and S1 = Q1 K_j^T
         //   warp 2: O0 += P0 V_j        warp 3: O1 += P1 V_j
-        // Each of the three warps releases a K/V stage once its own MMAs on it are done.
+        // Each of the three warps releases a K/V stage once its own MMAs on it are done (the S
+        // warp also on behalf of a PV warp with no work on the tile).
         bool ok = true;
         int it = 0;                  // K/V tiles consumed, over all items
         int n_item = 0;
@@ -320,7 +321,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         mma_commit(&sm.bar_s_full[t]);
                         ++ct[t];
                     }
-                    if (ok) mma_commit(&sm.bar_kv_empty[s]);
+                    if (ok) {
+                        mma_commit(&sm.bar_kv_empty[s]);
+                        // A PV warp with nothing to do on this tile leaves its release of stage s
+                        // to this warp: made here, after the stage's load was waited for, it can
+                        // only count towards this tile's phase.
+                        for (int t = 0; t < 2; ++t)
+                            if (j < lo[t] || j > hi[t]) mma_commit(&sm.bar_kv_empty[s]);
+                    }
                 }
                 if (ok) mma_commit(&sm.bar_q_empty[qbuf]);    // the item's Q buffer may be reloaded
                 ++n_item;
@@ -341,14 +349,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int lo = t ? lo1 : lo0, hi = t ? hi1 : hi0;
                 for (int j = lo0; ok && j <= hi1; ++j, ++it) {
                     const int s = it % kStages;
-                    if (j < lo || j > hi) {
-                        // Nothing of this warp reads stage s here.  Arrive only once the stage holds
-                        // this tile: an arrival made earlier could complete the stage's previous phase
-                        // while another warp's MMAs still read it.
-                        if (!(ok = mbar_wait(&sm.bar_k[s], (it / kStages) & 1, ac))) break;
-                        mbar_arrive(&sm.bar_kv_empty[s]);
-                        continue;
-                    }
+                    if (j < lo || j > hi) continue;      // the S warp releases stage s for this warp
                     const int i = j - lo;
                     if (!(ok = mbar_wait(&sm.bar_v[s], (it / kStages) & 1, ac))) break;
                     if (!(ok = mbar_wait(&sm.bar_p_full[t], ct & 1, ac))) break;
