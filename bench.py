@@ -465,10 +465,13 @@ def main():
         time.sleep(0.25)   # let the sampler start before the timed region
         barrier()
         with NvmlClockSampler(dev) as nclk:
+            host_s = 0.0
             for i in range(args.steps):
                 if flush is not None:
                     flush.zero_()
+                h0 = time.perf_counter()
                 step(evs[i])
+                host_s += time.perf_counter() - h0
             barrier()
     status = ga.gpt_attn_check(stream)
     if status != ga.GPT_ATTN_OK:
@@ -565,6 +568,9 @@ def main():
         "pct_of_peak": value / world / peaks["bf16_tflops"],
         "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": 4 * args.steps, "clocks": nclk.summary() or clk.summary(),
+        # CPU time to issue one step's four library calls (binding, C entry points, launches;
+        # the CUDA event records in between included)
+        "host_us_per_step": host_s / args.steps * 1e6,
     }
     print(json.dumps(line), flush=True)
     if dist is not None:
