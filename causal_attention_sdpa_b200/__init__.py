@@ -130,11 +130,12 @@ def _stream_handle(stream):
     import torch
     if stream is None:
         stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
 def _ptr(t):
-    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+    # A plain int: the c_void_p argtypes convert it (and None to NULL) without a wrapper object.
+    return t.data_ptr() if t is not None else None
 
 
 def _check_bf16(name, t, shape):
@@ -241,11 +242,24 @@ def _strides(t):
     return GptAttnStrides(t.stride(0), t.stride(1), t.stride(2))
 
 
+_STRIDES24 = ctypes.c_longlong * 24
+
+
 def _layout(**tensors):
-    lay = GptAttnLayout()
-    for n, t in tensors.items():
-        setattr(lay, n, _strides(t))
-    return lay
+    """A GptAttnLayout of the tensors' strides (given in the struct's order q, k, v, o, dO, dq, dk,
+    dv), or None when they are all contiguous [B, H, T, D] (the C default)."""
+    ts = list(tensors.values())
+    if all(t.is_contiguous() for t in ts):
+        return None
+    v = []
+    for t in ts:
+        st = t.stride()
+        v += (st[0], st[1], st[2])
+    return GptAttnLayout.from_buffer(_STRIDES24(*v))     # one flat copy; the struct keeps it alive
+
+
+def _byref(x):
+    return ctypes.byref(x) if x is not None else None
 
 
 def gpt_attn_fwd_ex(q, k, v, scale=None, window=0, head_windows=None, doc_start=None, o=None, lse=None,
@@ -266,7 +280,7 @@ def gpt_attn_fwd_ex(q, k, v, scale=None, window=0, head_windows=None, doc_start=
     m, keep = _mask(H, window, head_windows, doc_start)
     lay = _layout(q=q, k=k, v=v, o=o, dO=o, dq=o, dk=o, dv=o)
     rc = lib().gpt_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, D, float(scale),
-                               ctypes.byref(m), ctypes.byref(lay), _stream_handle(stream))
+                               ctypes.byref(m), _byref(lay), _stream_handle(stream))
     del keep
     if rc != GPT_ATTN_OK:
         raise GptAttnError(rc, "gpt_attn_fwd_ex")
@@ -294,7 +308,7 @@ def gpt_attn_bwd_ex(q, k, v, o, lse, dO, scale=None, window=0, head_windows=None
     m, keep = _mask(H, window, head_windows, doc_start)
     lay = _layout(q=q, k=k, v=v, o=o, dO=dO, dq=dq, dk=dk, dv=dv)
     rc = lib().gpt_attn_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk),
-                               _ptr(dv), B, H, T, D, float(scale), ctypes.byref(m), ctypes.byref(lay), _ptr(ws),
+                               _ptr(dv), B, H, T, D, float(scale), ctypes.byref(m), _byref(lay), _ptr(ws),
                                nbytes, _stream_handle(stream))
     del keep
     if rc != GPT_ATTN_OK:

@@ -16,7 +16,7 @@
 //                          stay in shared memory while the query tiles that see
 //                          them stream through a TMA ring (D=64: persistent CTAs
 //                          taking these units from a counter; D=128: one CTA per
-//                          unit).  Per query tile, five tcgen05 MMAs:
+//                          unit), in the list order of schedule.h.  Per query tile, five tcgen05 MMAs:
 //                            S^T  = K Q^T          (TMEM)
 //                            dP^T = V dO^T         (TMEM)
 //                            dV  += P^T dO         (P^T read from TMEM)
@@ -57,6 +57,7 @@ struct BwdParams {
     int T_pad;
     int BH;
     int n_tiles;
+    int tail;               // heads of the unit list's class-major tail (schedule.h)
     float scale_log2;       // scale * log2(e)
     float scale;
     uint64_t timeout_ns;
@@ -216,8 +217,8 @@ attn_bwd_serial_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const int lane = threadIdx.x & 31;
     // Blocks of one head are adjacent in launch order (its Q, dO and dQ rows stay in
     // L2 across its key tiles); key tile 0 sees the most query tiles and launches first.
-    const int bh = blockIdx.x / p.n_tiles;
-    const int kt = blockIdx.x % p.n_tiles;
+    int bh, kt;
+    list_item(blockIdx.x, p.BH, p.n_tiles, p.tail, bh, kt);   // unit list order of schedule.h
     const int k0 = kt * kTile;
     const int qt_lo = kt;
     const int W = mask.head_window(bh);

@@ -4,8 +4,9 @@
 // dS = P (dP - Delta), dK, dQ) and the same work unit: one (batch*head, 128-key
 // tile), whose K and V stay in shared memory while the query tiles that see it
 // stream past.  One CTA runs per SM and takes work units from a counter in the
-// workspace, in head-major order (the units of a head run close together, so its
-// Q, dO and dQ rows are served from L2).  K/V are double-buffered across units,
+// workspace, in the list order of schedule.h (head-major, so the units of a head
+// run close together and its Q, dO and dQ rows are served from L2; a tail that
+// ends with short units).  K/V are double-buffered across units,
 // so the next unit's loads and first scores overlap the end of the current one.
 //
 //   16 warps:
@@ -91,12 +92,12 @@ struct Bwd64Unit {
     int bh, kt, k0, qt_lo, n_q, W;
 };
 
-// Work unit u (head-major): head bh, key tile kt, and the n_q query tiles [kt, kt + n_q) that see it.
+// Work unit u of the list (schedule.h): head bh, key tile kt, and the n_q query tiles
+// [kt, kt + n_q) that see it.
 template <typename Mask>
 __device__ __forceinline__ Bwd64Unit bwd64_unit(int u, const BwdParams& p, const Mask& mask) {
     Bwd64Unit w;
-    w.bh = u / p.n_tiles;
-    w.kt = u % p.n_tiles;
+    list_item(u, p.BH, p.n_tiles, p.tail, w.bh, w.kt);
     w.W = mask.head_window(w.bh);
     w.n_q = bwd_last_tile(p, w.bh, w.kt, w.W) - w.kt + 1;
     w.k0 = w.kt * kTile;

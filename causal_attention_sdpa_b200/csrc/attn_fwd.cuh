@@ -7,15 +7,22 @@
 // when the max grows).  The mapping onto sm_100a is this file's own:
 //
 //   one work item = one (batch*head, 256-query block) = two 128-row Q tiles sharing
-//   every K/V tile it loads.  The kernel is persistent: each CTA (one per SM, as
-//   TMEM allows) runs a fixed sequence of items, and every barrier phase counts
-//   tiles over all the items a role has handled, so the next item's Q load and
-//   first scores overlap the current item's last tiles and epilogue.  Items go
-//   out in waves of whole heads (the 256-query blocks of a head run at the same
-//   time, so its K/V tiles come from HBM once and from L2 to the other blocks);
-//   from one wave to the next, the block length class each CTA gets rotates, so
-//   every CTA gets an even mix of long and short blocks.  12 warps:
-//     warp 0       TMA producer: Q0, Q1 once, then K_j / V_j through a ring
+//   every K/V tile it loads.  Only one block fits on an SM, and a block that starts
+//   does not stop after one item: the producer warp fetches item after item and passes
+//   each to the other roles through a two-slot ring in shared memory, and every
+//   barrier phase counts tiles over all the items a role has handled, so the next
+//   item's Q load and first scores overlap the current item's last tiles and epilogue.
+//   The items come in one of two orders (schedule.h):
+//     - on demand: the grid has one block per item, in list order (head-major, so the
+//       blocks of a head run at the same time and its K/V tiles come from HBM once and
+//       from L2 to the others; a tail that ends with short items); each running block
+//       takes the next item by cancelling, through cluster launch control, the launch
+//       of the first block that has not started;
+//     - static, for work of many full rounds: one block per SM, each running a fixed
+//       sequence of items in waves of whole heads, its block class rotating from one
+//       wave to the next.
+//   12 warps:
+//     warp 0       TMA producer and work-item fetcher: Q0, Q1 once, then K_j / V_j through a ring
 //     warp 1       TMEM allocator; issues S0 = Q0 K_j^T and S1 = Q1 K_j^T
 //     warps 2, 3   issue O0 += P0 V_j and O1 += P1 V_j (one MMA stream per warp)
 //     warps 4..7   softmax warpgroup of Q tile 0 (thread r owns query row r)
@@ -101,16 +108,36 @@ struct FwdParams {
     int BH;
     int n_tiles;          // ceil(T / 128)
     int n_blocks;         // ceil(n_tiles / 2): 256-query blocks per head
-    int heads_per_wave;   // the grid is heads_per_wave * n_blocks CTAs
-    int n_waves;          // ceil(BH / heads_per_wave)
+    int tail;             // heads of the item list's class-major tail (schedule.h)
+    int static_hpw;       // static order (schedule.h): heads per wave, and
+    int static_waves;     // waves (0: items taken from the list through cluster launch control)
     float scale_log2;     // scale * log2(e)
     uint64_t timeout_ns;
 };
 
-// Work item of CTA `cta` in wave `k` (schedule.h).
-__device__ __forceinline__ void fwd_item(const FwdParams& p, int cta, int k, int& bh, int& qb) {
-    fwd_item(p.heads_per_wave, p.n_blocks, p.BH, cta, k, bh, qb);
+// The work-item ring carries bh * n_blocks + qb (or -1: no more work).
+__device__ __forceinline__ int fwd_list_item(const FwdParams& p, int i) {
+    int bh, qb;
+    fwd_item(i, p.BH, p.n_blocks, p.tail, bh, qb);
+    return bh * p.n_blocks + qb;
 }
+
+// This block's static item after wave *k (advancing *k past it), or -1.
+__device__ __forceinline__ int fwd_next_static_item(const FwdParams& p, int& k) {
+    for (; k < p.static_waves; ++k) {
+        int bh, qb;
+        fwd_static_item(p.static_hpw, p.n_blocks, p.BH, blockIdx.x, k, bh, qb);
+        if (bh >= 0) {
+            ++k;
+            return bh * p.n_blocks + qb;
+        }
+    }
+    return -1;
+}
+
+// Roles that read each work item from the ring: the S warp, the two PV warps (one lane each) and
+// the eight softmax warps (one arrival per warp).
+constexpr int kFwdItemReaders = 3 + 8;
 
 // Key tiles [lo, hi] of query tile qt of head bh with window W.
 template <typename Mask>
@@ -151,6 +178,11 @@ struct FwdSmem {
     uint64_t bar_ostage_free[2];  // warpgroup t's previous O tile store has read its staging buffer
     uint64_t bar_ostage_full[2];  // warpgroup t has staged its O tile
     uint64_t bar_drain;
+    uint64_t bar_item_full[2];    // work-item ring: slot written by the producer
+    uint64_t bar_item_empty[2];   // slot read by every role
+    uint64_t bar_clc;             // cluster launch control response landed
+    alignas(16) uint32_t clc_resp[4];
+    int item[2];                  // work item, or -1 when there is none left
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -180,7 +212,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int cta = blockIdx.x;
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < kQBufs; ++b) {
@@ -202,6 +233,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&sm.bar_ostage_full[t], 128);
         }
         mbar_init(&sm.bar_drain, 3);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.bar_item_full[b], 1);
+            mbar_init(&sm.bar_item_empty[b], kFwdItemReaders);
+        }
+        mbar_init(&sm.bar_clc, 1);
         sm.abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -215,6 +251,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const AbortCtl ac{&sm.abort_flag, p.timeout_ns};
+    // Work item n of this block for a single-lane role: waits for ring slot n % 2, reads it,
+    // releases it.
+    auto read_item = [&](int n, int& i) -> bool {
+        const int slot = n & 1;
+        if (!mbar_wait(&sm.bar_item_full[slot], (n >> 1) & 1, ac)) return false;
+        i = *reinterpret_cast<volatile int*>(&sm.item[slot]);
+        mbar_arrive(&sm.bar_item_empty[slot]);
+        return true;
+    };
     // Launched with 168 registers per thread (384 x 168 = 64512): warpgroup 0
     // (producer, MMA, two idle warps) drops to 64, the softmax warpgroups take 216.
     // 128 x 64 + 256 x 216 = 63488 <= 64512.
@@ -230,11 +275,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_prefetch_desc(&tm_v);
             int it = 0;              // K/V tiles loaded, over all items
             int n_item = 0;          // items whose Q was loaded
+            int n_clc = 0;           // launch-control responses received
+            bool clc_pending = false;
             bool ok = true;
-            for (int k = 0; ok && k < p.n_waves; ++k) {
-                int bh, qb;
-                fwd_item(p, cta, k, bh, qb);
-                if (bh < 0) continue;
+            const bool dynamic = p.static_waves == 0;
+            int k_static = 0;        // static order: next wave
+            // This block's own item first.
+            int cur = dynamic ? fwd_list_item(p, blockIdx.x) : fwd_next_static_item(p, k_static);
+            for (int n = 0; ok; ++n) {
+                const int slot = n & 1;
+                if (n >= 2 && !(ok = mbar_wait(&sm.bar_item_empty[slot], ((n >> 1) - 1) & 1, ac))) break;
+                *reinterpret_cast<volatile int*>(&sm.item[slot]) = cur;
+                mbar_arrive(&sm.bar_item_full[slot]);
+                if (cur < 0) break;
+                if (dynamic) {
+                    // Ask now for the item after this one (the item of the first block that has not
+                    // started); the answer is read once this item's loads are out.
+                    mbar_arrive_expect_tx(&sm.bar_clc, 16);
+                    clc_try_cancel(sm.clc_resp, &sm.bar_clc);
+                    clc_pending = true;
+                }
+                const int bh = cur / p.n_blocks, qb = cur % p.n_blocks;
                 const int W = mask.head_window(bh);
                 int lo0, hi0, lo1, hi1;
                 fwd_tile_range(p, mask, bh, W, 2 * qb, lo0, hi0);
@@ -262,7 +323,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int b = 0; b < kBoxes; ++b)
                         tma_load_4d(sm.v[s] + b * 16384, &tm_v, &sm.bar_v[s], b * 64, j * kTile, hh, bb);
                 }
+                if (!ok) break;
+                if (!dynamic) {
+                    cur = fwd_next_static_item(p, k_static);
+                    continue;
+                }
+                if (!(ok = mbar_wait(&sm.bar_clc, n_clc & 1, ac))) break;
+                clc_pending = false;
+                ++n_clc;
+                const int b = clc_cancelled_block(sm.clc_resp);
+                cur = b < 0 ? -1 : fwd_list_item(p, b);
             }
+            // A request still out when the block gave up must land before the block exits.
+            if (clc_pending) mbar_wait_drain(&sm.bar_clc, n_clc & 1, p.timeout_ns);
             if (sm.abort_flag) {
                 // Let every load already issued land before the CTA exits.
                 for (int r = (n_item > kQBufs ? n_item - kQBufs : 0); r < n_item; ++r)
@@ -286,10 +359,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         int n_item = 0;
         if (warp == 1) {
             int ct[2] = {0, 0};      // S tiles issued per warpgroup, over all items
-            for (int k = 0; ok && k < p.n_waves; ++k) {
-                int bh, qb;
-                fwd_item(p, cta, k, bh, qb);
-                if (bh < 0) continue;
+            for (int n = 0; ok; ++n) {
+                int cur;
+                if (!(ok = read_item(n, cur)) || cur < 0) break;
+                const int bh = cur / p.n_blocks, qb = cur % p.n_blocks;
                 const int W = mask.head_window(bh);
                 int lo[2], hi[2];
                 fwd_tile_range(p, mask, bh, W, 2 * qb, lo[0], hi[0]);
@@ -338,10 +411,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t col_o = t ? C::kColO1 : C::kColO0;
             const uint32_t col_p = t ? C::kColP1 : C::kColP0;
             int ct = 0;              // PV tiles issued, over all items
-            for (int k = 0; ok && k < p.n_waves; ++k) {
-                int bh, qb;
-                fwd_item(p, cta, k, bh, qb);
-                if (bh < 0) continue;
+            for (int n = 0; ok; ++n) {
+                int cur;
+                if (!(ok = read_item(n, cur)) || cur < 0) break;
+                const int bh = cur / p.n_blocks, qb = cur % p.n_blocks;
                 const int W = mask.head_window(bh);
                 int lo0, hi0, lo1, hi1;
                 fwd_tile_range(p, mask, bh, W, 2 * qb, lo0, hi0);
@@ -389,10 +462,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         int ct = 0;                  // tiles of this warpgroup, over all items
         int n_items = 0;
         const bool o_issuer = wq == 0 && lane == 0;   // issues this warpgroup's O tile stores
-        for (int k = 0; ok && k < p.n_waves; ++k) {
-            int bh, qb;
-            fwd_item(p, cta, k, bh, qb);
-            if (bh < 0) continue;
+        for (int n = 0; ok; ++n) {
+            const int slot = n & 1;
+            if (!warp_wait(&sm.bar_item_full[slot], (n >> 1) & 1, ac)) { ok = false; break; }
+            const int cur = *reinterpret_cast<volatile int*>(&sm.item[slot]);
+            __syncwarp();                                // every lane has read the slot
+            if (lane == 0) mbar_arrive(&sm.bar_item_empty[slot]);
+            if (cur < 0) break;
+            const int bh = cur / p.n_blocks, qb = cur % p.n_blocks;
             const int qt = 2 * qb + t;
             const int i_abs = qt * kTile + row;
             const int W = mask.head_window(bh);

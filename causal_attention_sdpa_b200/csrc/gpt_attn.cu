@@ -9,6 +9,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "attn_bwd.cuh"
 #include "attn_bwd_d64.cuh"
@@ -142,7 +143,26 @@ int check_shape(int B, int H, int T, int D) {
 
 template <typename Kern>
 bool set_smem(Kern k, size_t bytes) {
-    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+    // The attribute is a per-function setting: raise it once per kernel and device (and again only
+    // for a larger size) instead of paying a driver call on every launch.
+    struct Entry { const void* fn; int dev; size_t bytes; };
+    static std::mutex mu;
+    static std::vector<Entry> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const void* fn = reinterpret_cast<const void*>(k);
+    std::lock_guard<std::mutex> g(mu);
+    for (auto& e : done)
+        if (e.fn == fn && e.dev == dev) {
+            if (e.bytes >= bytes) return true;
+            if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+                return false;
+            e.bytes = bytes;
+            return true;
+        }
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) return false;
+    done.push_back({fn, dev, bytes});
+    return true;
 }
 
 int sm_count();
@@ -193,14 +213,21 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.n_blocks = (p.n_tiles + 1) / 2;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = wait_timeout_ns();
-    // D = 64: persistent grid, waves of whole heads, heads_per_wave * n_blocks CTAs, at most one
-    // per SM (TMEM holds one CTA's accumulators) unless a single head has more blocks than the GPU
-    // has SMs.  D = 128: one item per CTA (a single wave of all heads): its Q tiles cannot be
-    // double-buffered next to the K/V ring, so a CTA would wait for each new item's Q.
-    fwd_grid(sm_count(), p.n_blocks, BH, D == 64, p.heads_per_wave, p.n_waves);
-    const int hpw = p.heads_per_wave;
+    // Work order (schedule.h): static waves with one block per SM when they make enough full
+    // rotations (D = 64), else one block per item, the blocks that start taking the items of
+    // those that have not through cluster launch control.
+    const int sms = sm_count();
+    p.tail = tail_heads(BH, p.n_blocks, sms);
+    p.static_hpw = 0;
+    p.static_waves = 0;
+    int hpw, waves;
+    const bool stat = D == 64 && fwd_static_grid(sms, p.n_blocks, BH, hpw, waves);
+    if (stat) {
+        p.static_hpw = hpw;
+        p.static_waves = waves;
+    }
     const size_t smem = sizeof(FwdSmem<D>) + 1024;
-    const unsigned grid = (unsigned)((long long)hpw * p.n_blocks);
+    const unsigned grid = stat ? (unsigned)(hpw * p.n_blocks) : (unsigned)((long long)BH * p.n_blocks);
     if (plain_window(mask)) {
         // Causal or one window for every head: the instantiation without per-head or document data.
         if (!set_smem(attn_fwd_kernel<D, WindowMask>, smem)) return GPT_ATTN_ERR_CUDA;
@@ -297,6 +324,7 @@ int launch_bwd_grads(const void* q, const void* k, const void* v, const void* do
     p.T_pad = w.T_pad;
     p.BH = BH;
     p.n_tiles = w.n_tiles;
+    p.tail = tail_heads(BH, p.n_tiles, sm_count());
     p.lower2 = mask.doc_start ? w.lower2 : nullptr;
     p.last_qt = mask.doc_start ? w.last_qt : nullptr;
     p.scale_log2 = scale * 1.4426950408889634f;

@@ -1,6 +1,6 @@
 // Work decomposition of the attention kernels, as plain integer code: which key tiles a query
-// tile sees, which query tiles a key tile reaches, the forward kernel's persistent item order and
-// the backward kernel's work units.  nvcc compiles it into the kernels and the host launcher; the
+// tile sees, which query tiles a key tile reaches, and the order in which the work items of both
+// passes go to the SMs.  nvcc compiles it into the kernels and the host launcher; the
 // CPU tests compile the same header with a host compiler and check it against brute force.
 //
 // Visibility follows the masked softmax of the causal attention definition: query i sees key j
@@ -66,23 +66,64 @@ GPT_ATTN_HD int bwd_last_query_tile_lb(int kt, int n_tiles, LowerOfTile lower_of
     return qt;
 }
 
-// Forward grid.  A work item is one (head, 256-query block); n_blocks = ceil(n_tiles / 2) per
-// head.  Persistent (D = 64): waves of whole heads, heads_per_wave * n_blocks CTAs, at most one
-// per SM unless a single head has more blocks than the GPU has SMs.  D = 128: one item per CTA
-// (a single wave of all heads).
-GPT_ATTN_HD void fwd_grid(int sms, int n_blocks, int BH, bool persistent, int& heads_per_wave, int& n_waves) {
-    int hpw = persistent ? sms / n_blocks : BH;
+// Work order of both passes.  Every pass splits into work items of one head each, n_cls of
+// them per head (the forward: 256-query blocks; the backward: 128-key tiles), and the items go
+// to the SMs in a fixed list order, each SM taking the next item when it is ready for one (the
+// forward kernel through cluster launch control, the backward kernel from a counter; the
+// forward kernel also has a static order, below).  The
+// items of one head should run at the same time, so that what they share (K/V in the forward;
+// Q, dO and the dQ accumulator in the backward) is read from HBM once and from L2 by the
+// others while it is still there: the list is head-major, each head's items longest first
+// (class 0: the last query block in the forward, the first key tile in the backward).  Taken
+// that way, though, the list would end with the long items of the last heads while the other
+// SMs run dry; so the last `tail` heads go class-major instead (all their class-0 items, then
+// all their class-1 items, ...), and the list ends with short items.
+
+// Heads of the class-major tail: enough for the tail to hold two items per SM.
+GPT_ATTN_HD int tail_heads(int BH, int n_cls, int sms) {
+    const int t = (2 * sms + n_cls - 1) / n_cls;
+    return t < BH ? t : BH;
+}
+
+// Item i of the list (0 <= i < BH * n_cls) whose last `tail` heads go class-major.  Returns
+// head and class.
+GPT_ATTN_HD void list_item(int i, int BH, int n_cls, int tail, int& bh, int& cls) {
+    const int head_major = (BH - tail) * n_cls;     // items before the tail
+    if (i < head_major) {
+        bh = i / n_cls;
+        cls = i % n_cls;
+    } else {
+        const int l = i - head_major;
+        cls = l / tail;
+        bh = BH - tail + l % tail;
+    }
+}
+
+// The forward kernel has a second, static order for work that comes in many full rounds: items
+// go out in waves of whole heads, heads_per_wave * n_blocks blocks, one per SM, and from one wave
+// to the next the block class each block gets rotates, so that over n_blocks waves every block
+// runs every class once.  Measured on the GPT-2 shapes this beats taking items on demand when
+// the waves make at least kStaticCycles full rotations; with fewer, the partial rotation leaves
+// some SMs with much more work than others, and the list above is used instead.
+constexpr int kStaticCycles = 4;
+
+// Static forward grid for n_blocks blocks per head: heads_per_wave and n_waves, and whether the
+// static order applies at all.
+GPT_ATTN_HD bool fwd_static_grid(int sms, int n_blocks, int BH, int& heads_per_wave, int& n_waves) {
+    int hpw = sms / n_blocks;
     if (hpw < 1) hpw = 1;
     if (hpw > BH) hpw = BH;
     heads_per_wave = hpw;
     n_waves = (BH + hpw - 1) / hpw;
+    return hpw * n_blocks <= sms && n_waves >= kStaticCycles * n_blocks;
 }
 
-// Work item of CTA `cta` in wave `k`: head bh (or -1 when the wave has no item for it) and
-// 256-query block qb.  Slot s of a wave holds block class s / heads_per_wave (longest first)
-// of head s % heads_per_wave; a CTA's slot moves on by heads_per_wave each wave, so each CTA
-// gets an even mix of long and short blocks while the blocks of a head run at the same time.
-GPT_ATTN_HD void fwd_item(int heads_per_wave, int n_blocks, int BH, int cta, int k, int& bh, int& qb) {
+// Static item of block `cta` in wave k: head bh (or -1 when the wave has none for it) and block
+// qb.  Slot s of a wave holds block class s / heads_per_wave (longest first) of head
+// s % heads_per_wave; a block's slot moves on by heads_per_wave each wave, so each block keeps
+// to the same head position and cycles through the classes, while the blocks of a head run at
+// the same time.
+GPT_ATTN_HD void fwd_static_item(int heads_per_wave, int n_blocks, int BH, int cta, int k, int& bh, int& qb) {
     const int G = heads_per_wave * n_blocks;
     const int slot = (int)(((long long)cta + (long long)heads_per_wave * k) % G);
     bh = heads_per_wave * k + slot % heads_per_wave;
@@ -90,11 +131,18 @@ GPT_ATTN_HD void fwd_item(int heads_per_wave, int n_blocks, int BH, int cta, int
     if (bh >= BH) bh = -1;
 }
 
-// Backward work unit u of the persistent kernel: head bh, key tile kt, and the n_q query tiles
-// [kt, kt + n_q) that see it.  Units are numbered head-major.
-GPT_ATTN_HD void bwd_unit(int u, int n_tiles, int window, int& bh, int& kt, int& n_q) {
-    bh = u / n_tiles;
-    kt = u % n_tiles;
+// Forward item i: head bh and 256-query block qb (class 0 = the last block, the longest under
+// a causal mask).
+GPT_ATTN_HD void fwd_item(int i, int BH, int n_blocks, int tail, int& bh, int& qb) {
+    int cls;
+    list_item(i, BH, n_blocks, tail, bh, cls);
+    qb = n_blocks - 1 - cls;
+}
+
+// Backward work unit u: head bh, key tile kt (class 0 = key tile 0, seen by the most query
+// tiles), and the n_q query tiles [kt, kt + n_q) that see it under a window (no document mask).
+GPT_ATTN_HD void bwd_unit(int u, int BH, int n_tiles, int tail, int window, int& bh, int& kt, int& n_q) {
+    list_item(u, BH, n_tiles, tail, bh, kt);
     n_q = bwd_last_query_tile(kt, n_tiles, window) - kt + 1;
 }
 

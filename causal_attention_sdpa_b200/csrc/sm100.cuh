@@ -146,6 +146,38 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- cluster launch control
+// A running block asks the hardware to cancel the launch of a grid block that has not started yet
+// and takes over its work.  The 16-byte response lands in shared memory at `resp` (16-byte
+// aligned) and completes 16 bytes of transactions on `bar`, which the caller armed with
+// mbar_arrive_expect_tx.  Once a request has come back empty no further request may be made.
+__device__ __forceinline__ void clc_try_cancel(void* resp, uint64_t* bar) {
+    asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];"
+                 ::"r"(smem_u32(resp)), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// x index of the block a completed response cancelled, or -1 if it cancelled none (every block
+// of the grid has started).  Orders the read before a later request rewrites the buffer.
+__device__ __forceinline__ int clc_cancelled_block(const void* resp) {
+    uint32_t ok, x;
+    asm volatile(
+        "{\n\t"
+        ".reg .pred p;\n\t"
+        ".reg .b128 r;\n\t"
+        "mov.u32 %1, 0;\n\t"
+        "ld.shared.b128 r, [%2];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t"
+        "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t"
+        "}"
+        : "=r"(ok), "=r"(x)
+        : "r"(smem_u32(resp))
+        : "memory");
+    fence_proxy_async_smem();
+    return ok ? (int)x : -1;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
