@@ -115,24 +115,21 @@ struct FwdParams {
     uint64_t timeout_ns;
 };
 
-// The work-item ring carries bh * n_blocks + qb (or -1: no more work).
-__device__ __forceinline__ int fwd_list_item(const FwdParams& p, int i) {
-    int bh, qb;
+// Item i of the list: head bh and 256-query block qb.
+__device__ __forceinline__ void fwd_list_item(const FwdParams& p, int i, int& bh, int& qb) {
     fwd_item(i, p.BH, p.n_blocks, p.tail, bh, qb);
-    return bh * p.n_blocks + qb;
 }
 
-// This block's static item after wave *k (advancing *k past it), or -1.
-__device__ __forceinline__ int fwd_next_static_item(const FwdParams& p, int& k) {
+// This block's static item after wave *k (advancing *k past it); bh = -1 when there is none.
+__device__ __forceinline__ void fwd_next_static_item(const FwdParams& p, int& k, int& bh, int& qb) {
+    bh = -1;
     for (; k < p.static_waves; ++k) {
-        int bh, qb;
         fwd_static_item(p.static_hpw, p.n_blocks, p.BH, blockIdx.x, k, bh, qb);
         if (bh >= 0) {
             ++k;
-            return bh * p.n_blocks + qb;
+            return;
         }
     }
-    return -1;
 }
 
 // Roles that read each work item from the ring: the S warp, the two PV warps (one lane each) and
@@ -182,7 +179,8 @@ struct FwdSmem {
     uint64_t bar_item_empty[2];   // slot read by every role
     uint64_t bar_clc;             // cluster launch control response landed
     alignas(16) uint32_t clc_resp[4];
-    int item[2];                  // work item, or -1 when there is none left
+    int item_bh[2];               // work item: head, or -1 when there is none left,
+    int item_qb[2];               // and 256-query block
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -253,20 +251,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const AbortCtl ac{&sm.abort_flag, p.timeout_ns};
     // Work item n of this block for a single-lane role: waits for ring slot n % 2, reads it,
     // releases it.
-    auto read_item = [&](int n, int& i) -> bool {
+    auto read_item = [&](int n, int& bh, int& qb) -> bool {
         const int slot = n & 1;
         if (!mbar_wait(&sm.bar_item_full[slot], (n >> 1) & 1, ac)) return false;
-        i = *reinterpret_cast<volatile int*>(&sm.item[slot]);
+        bh = *reinterpret_cast<volatile int*>(&sm.item_bh[slot]);
+        qb = *reinterpret_cast<volatile int*>(&sm.item_qb[slot]);
         mbar_arrive(&sm.bar_item_empty[slot]);
         return true;
     };
     // Launched with 168 registers per thread (384 x 168 = 64512): warpgroup 0
-    // (producer, MMA, two idle warps) drops to 64, the softmax warpgroups take 216.
-    // 128 x 64 + 256 x 216 = 63488 <= 64512.
+    // (producer, MMA) drops to 56, the softmax warpgroups take 224:
+    // 128 x 56 + 256 x 224 = 64512.  The softmax pass runs faster with 224 than with
+    // 216 (more exponentials in flight); 232 gains nothing more.
     // Each role's code sits under its own setmaxnreg so the compiler allocates it
     // with that role's budget.
     if (warp < 4) {
-        regs_dec<64>();
+        regs_dec<56>();
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -281,13 +281,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const bool dynamic = p.static_waves == 0;
             int k_static = 0;        // static order: next wave
             // This block's own item first.
-            int cur = dynamic ? fwd_list_item(p, blockIdx.x) : fwd_next_static_item(p, k_static);
+            int bh, qb;
+            if (dynamic)
+                fwd_list_item(p, blockIdx.x, bh, qb);
+            else
+                fwd_next_static_item(p, k_static, bh, qb);
             for (int n = 0; ok; ++n) {
                 const int slot = n & 1;
                 if (n >= 2 && !(ok = mbar_wait(&sm.bar_item_empty[slot], ((n >> 1) - 1) & 1, ac))) break;
-                *reinterpret_cast<volatile int*>(&sm.item[slot]) = cur;
+                *reinterpret_cast<volatile int*>(&sm.item_bh[slot]) = bh;
+                *reinterpret_cast<volatile int*>(&sm.item_qb[slot]) = qb;
                 mbar_arrive(&sm.bar_item_full[slot]);
-                if (cur < 0) break;
+                if (bh < 0) break;
                 if (dynamic) {
                     // Ask now for the item after this one (the item of the first block that has not
                     // started); the answer is read once this item's loads are out.
@@ -295,7 +300,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     clc_try_cancel(sm.clc_resp, &sm.bar_clc);
                     clc_pending = true;
                 }
-                const int bh = cur / p.n_blocks, qb = cur % p.n_blocks;
                 const int W = mask.head_window(bh);
                 int lo0, hi0, lo1, hi1;
                 fwd_tile_range(p, mask, bh, W, 2 * qb, lo0, hi0);
@@ -325,14 +329,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 if (!ok) break;
                 if (!dynamic) {
-                    cur = fwd_next_static_item(p, k_static);
+                    fwd_next_static_item(p, k_static, bh, qb);
                     continue;
                 }
                 if (!(ok = mbar_wait(&sm.bar_clc, n_clc & 1, ac))) break;
                 clc_pending = false;
                 ++n_clc;
                 const int b = clc_cancelled_block(sm.clc_resp);
-                cur = b < 0 ? -1 : fwd_list_item(p, b);
+                if (b < 0)
+                    bh = -1;
+                else
+                    fwd_list_item(p, b, bh, qb);
             }
             // A request still out when the block gave up must land before the block exits.
             if (clc_pending) mbar_wait_drain(&sm.bar_clc, n_clc & 1, p.timeout_ns);
@@ -360,9 +367,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (warp == 1) {
             int ct[2] = {0, 0};      // S tiles issued per warpgroup, over all items
             for (int n = 0; ok; ++n) {
-                int cur;
-                if (!(ok = read_item(n, cur)) || cur < 0) break;
-                const int bh = cur / p.n_blocks, qb = cur % p.n_blocks;
+                int bh, qb;
+                if (!(ok = read_item(n, bh, qb)) || bh < 0) break;
                 const int W = mask.head_window(bh);
                 int lo[2], hi[2];
                 fwd_tile_range(p, mask, bh, W, 2 * qb, lo[0], hi[0]);
@@ -412,9 +418,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t col_p = t ? C::kColP1 : C::kColP0;
             int ct = 0;              // PV tiles issued, over all items
             for (int n = 0; ok; ++n) {
-                int cur;
-                if (!(ok = read_item(n, cur)) || cur < 0) break;
-                const int bh = cur / p.n_blocks, qb = cur % p.n_blocks;
+                int bh, qb;
+                if (!(ok = read_item(n, bh, qb)) || bh < 0) break;
                 const int W = mask.head_window(bh);
                 int lo0, hi0, lo1, hi1;
                 fwd_tile_range(p, mask, bh, W, 2 * qb, lo0, hi0);
@@ -448,7 +453,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     }
     } else {
-        regs_inc<216>();
+        regs_inc<224>();
         // ------------------------------------------------------------ softmax warpgroups
         const int t = (warp - 4) >> 2;               // Q tile of this warpgroup
         const int wq = warp & 3;                     // TMEM lane quarter this warp may access
@@ -465,11 +470,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int n = 0; ok; ++n) {
             const int slot = n & 1;
             if (!warp_wait(&sm.bar_item_full[slot], (n >> 1) & 1, ac)) { ok = false; break; }
-            const int cur = *reinterpret_cast<volatile int*>(&sm.item[slot]);
+            const int bh = *reinterpret_cast<volatile int*>(&sm.item_bh[slot]);
+            const int qb = *reinterpret_cast<volatile int*>(&sm.item_qb[slot]);
             __syncwarp();                                // every lane has read the slot
             if (lane == 0) mbar_arrive(&sm.bar_item_empty[slot]);
-            if (cur < 0) break;
-            const int bh = cur / p.n_blocks, qb = cur % p.n_blocks;
+            if (bh < 0) break;
             const int qt = 2 * qb + t;
             const int i_abs = qt * kTile + row;
             const int W = mask.head_window(bh);

@@ -125,7 +125,7 @@ GPT_ATTN_HD bool fwd_static_grid(int sms, int n_blocks, int BH, int& heads_per_w
 // the same time.
 GPT_ATTN_HD void fwd_static_item(int heads_per_wave, int n_blocks, int BH, int cta, int k, int& bh, int& qb) {
     const int G = heads_per_wave * n_blocks;
-    const int slot = (int)(((long long)cta + (long long)heads_per_wave * k) % G);
+    const int slot = (cta + heads_per_wave * (k % n_blocks)) % G;   // hpw * k mod G cycles with k mod n_blocks
     bh = heads_per_wave * k + slot % heads_per_wave;
     qb = n_blocks - 1 - slot / heads_per_wave;
     if (bh >= BH) bh = -1;
