@@ -164,6 +164,28 @@ def test_outputs_fully_written(ga):
         assert torch.isfinite(t).all()
 
 
+@pytest.mark.parametrize("B,H,T,D,W", [(2, 3, 700, 64, 0), (1, 4, 1024, 64, 300), (2, 2, 333, 128, 0)])
+def test_staged_backward(ga, B, H, T, D, W):
+    """The three stages called one by one (delta, grads, dQ conversion) against the oracle and
+    against the one-call backward."""
+    s = D ** -0.5
+    q, k, v, do = make_inputs(B, H, T, D, seed=11)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = ga.gpt_attn_fwd(qd, kd, vd, scale=s, window=W)
+    ws = torch.empty(ga.gpt_attn_bwd_workspace_bytes(B, H, T, D), dtype=torch.uint8, device="cuda")
+    dq, dk, dv = (torch.full_like(qd, float("nan")) for _ in range(3))
+    ga.gpt_attn_bwd_delta(o, lse, dod, ws)
+    ga.gpt_attn_bwd_grads(qd, kd, vd, dod, dk, dv, ws, scale=s, window=W)
+    ga.gpt_attn_bwd_dq_convert(dq, ws, scale=s)
+    assert ga.gpt_attn_check() == ga.GPT_ATTN_OK
+    got = {"o": o.float().cpu(), "lse": lse.float().cpu(), "dq": dq.float().cpu(), "dk": dk.float().cpu(),
+           "dv": dv.float().cpu()}
+    compare(got, run_oracle(q, k, v, do, s, W), label="staged")
+    dq1, dk1, dv1 = ga.gpt_attn_bwd(qd, kd, vd, o, lse, dod, scale=s, window=W)
+    assert torch.equal(dk, dk1) and torch.equal(dv, dv1)
+    assert (dq.float() - dq1.float()).abs().max().item() <= 2 ** -6 * dq.float().abs().max().item()
+
+
 def test_forward_is_deterministic(ga):
     q, k, v, do = (t.cuda() for t in make_inputs(2, 4, 1024, 64, seed=6))
     o1, l1 = ga.gpt_attn_fwd(q, k, v)
