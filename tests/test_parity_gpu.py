@@ -118,21 +118,24 @@ def test_odd_shapes(ga, B, H, T, D, W, s):
     compare(got, ref, label=f"B{B}H{H}T{T}D{D}W{W}")
 
 
-# Shapes whose D = 64 launches put several work items on every CTA: the forward runs 3-7 waves
-# of whole heads and the backward 5-12 work units per CTA, so the barrier phases, Q-buffer reuse
+# Shapes whose launches put several work items on every CTA, so the barrier phases, Q-buffer reuse
 # and K/V double buffering carried from one item to the next are exercised on ragged last tiles
-# (T not a multiple of 128) and under windows (varying numbers of key tiles per query block and
-# of query tiles per key tile).  Every element of every head is compared with the oracle.
+# (T not a multiple of 128) and under windows (varying numbers of key tiles per query block and of
+# query tiles per key tile).  The forward takes its items on demand through cluster launch control
+# except where the static rotation has at least four full rounds (the B=48 case: 16 waves of 37
+# heads); the backward takes 5-12 work units per CTA from its list.  Every element of every head is
+# compared with the oracle.
 MULTI_ITEM = [
     # (B, H, T, D, window, scale)
-    (8, 12, 1000, 64, 0, 0.125),      # 3 forward waves, 768 backward units, ragged tail
+    (8, 12, 1000, 64, 0, 0.125),      # 384 forward items on demand, 768 backward units, ragged tail
     (8, 12, 1000, 64, 200, 0.125),    # same, windowed
-    (16, 12, 1024, 64, 256, 0.125),   # 6 waves, 1536 units, window of two tiles
-    (4, 40, 777, 64, 333, 0.125),     # 5 waves, 1120 units, ragged and windowed
-    (24, 8, 1100, 64, 1, 0.125),      # 7 waves, 1728 units, every query sees only itself
+    (16, 12, 1024, 64, 256, 0.125),   # 768 items, 1536 units, window of two tiles
+    (4, 40, 777, 64, 333, 0.125),     # 640 items, 1120 units, ragged and windowed
+    (24, 8, 1100, 64, 1, 0.125),      # 960 items, 1728 units, every query sees only itself
+    (48, 12, 1000, 64, 200, 0.125),   # static forward order (16 waves), ragged and windowed
+    (4, 8, 2500, 64, 700, 0.125),     # 10 blocks per head, ~2 items per CTA, ragged and windowed
     (2, 3, 700, 128, 1, 0.12),        # D = 128 with window 1
 ]
-
 
 @pytest.mark.parametrize("B,H,T,D,W,s", MULTI_ITEM, ids=[f"B{c[0]}H{c[1]}T{c[2]}D{c[3]}W{c[4]}" for c in MULTI_ITEM])
 def test_multi_item_parity(ga, B, H, T, D, W, s):
