@@ -448,10 +448,21 @@ int prologue_strides(Strides* out, const gpt_attn_strides* in, int n, int H, int
 
 int launch_prologue(bool backward, const PrologueParams& p, int D, cudaStream_t st) {
     // persistent: 2 blocks per SM for each of q and k, all resident at once (4 x 256 threads of
-    // at most 64 registers)
-    const long long rows_per_block = kPrologueThreads / (D / 16);
-    const long long need = (p.rows + rows_per_block - 1) / rows_per_block;
+    // at most 64 registers); a lane group takes a row, or a whole token for token-major inputs
+    const long long per_block = kPrologueThreads / (D / 16);
+    const long long units = p.token_major ? p.rows / p.H : p.rows;
+    const long long need = (units + per_block - 1) / per_block;
     const dim3 grid((unsigned)std::min<long long>(need, 2LL * sm_count()), 2);
+    if (p.token_major) {
+        if (backward) {
+            if (D == 64) qk_prologue_bwd_tok_kernel<64><<<grid, 256, 0, st>>>(p);
+            else qk_prologue_bwd_tok_kernel<128><<<grid, 256, 0, st>>>(p);
+        } else {
+            if (D == 64) qk_prologue_fwd_tok_kernel<64><<<grid, 256, 0, st>>>(p);
+            else qk_prologue_fwd_tok_kernel<128><<<grid, 256, 0, st>>>(p);
+        }
+        return cudaGetLastError() == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_CUDA;
+    }
     if (backward) {
         if (D == 64) qk_prologue_bwd_kernel<64><<<grid, 256, 0, st>>>(p);
         else qk_prologue_bwd_kernel<128><<<grid, 256, 0, st>>>(p);
@@ -642,7 +653,7 @@ int gpt_attn_qk_prologue_fwd(const void* q_raw, const void* k_raw, void* q_out, 
     p.H = H;
     p.T = T;
     p.rows = (long long)B * H * T;
-    p.token_major = st[0].t < st[0].h ? 1 : 0;    // walk rows in q_raw's memory order
+    p.token_major = st[0].h < st[0].t ? 1 : 0;    // heads of a token adjacent: walk rows token by token
     p.norm = qk_norm ? 1 : 0;
     p.base = rope_base;
     return launch_prologue(false, p, D, static_cast<cudaStream_t>(stream));
@@ -670,7 +681,7 @@ int gpt_attn_qk_prologue_bwd(const void* q_raw, const void* k_raw, const void* d
     p.H = H;
     p.T = T;
     p.rows = (long long)B * H * T;
-    p.token_major = st[0].t < st[0].h ? 1 : 0;    // walk rows in q_raw's memory order
+    p.token_major = st[0].h < st[0].t ? 1 : 0;    // heads of a token adjacent: walk rows token by token
     p.norm = qk_norm ? 1 : 0;
     p.base = rope_base;
     return launch_prologue(true, p, D, static_cast<cudaStream_t>(stream));

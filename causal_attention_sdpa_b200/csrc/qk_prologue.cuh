@@ -245,4 +245,148 @@ qk_prologue_bwd_kernel(const PrologueParams p) {
     }
 }
 
+// Token-major inputs (the q and k of a fused [B, T, 3, H, D] projection): the H heads of a token
+// are adjacent in memory and share their rotation angles, so a lane group takes a whole token, works
+// out its 8 angles once, and runs the token's heads two at a time, both heads' loads issued before
+// any arithmetic.  Same results as the kernels above (the same operations on each row).
+template <int D>
+__global__ void __launch_bounds__(kPrologueThreads, 4)
+qk_prologue_fwd_tok_kernel(const PrologueParams p) {
+    constexpr int G = D / 16, H2 = D / 2, kGroups = kPrologueThreads / G;
+    constexpr int UH = 1;                            // heads per batch of loads
+    const int which = blockIdx.y;
+    const int j = threadIdx.x % G;
+    __shared__ double rev[D / 2];
+    prologue_rev_per_token<D>(p.base, rev);
+    const __nv_bfloat16* xb = p.x[which];
+    __nv_bfloat16* yb = p.out[which];
+    const Strides xs = p.xs[which], ys = p.outs[which];
+    const long long n_tok = p.rows / p.H;            // B * T
+    // warp-uniform loop bound (the warp's first token), as in the row kernels
+    for (long long tok0 = (long long)blockIdx.x * kGroups + (threadIdx.x & ~31) / G; tok0 < n_tok;
+         tok0 += (long long)gridDim.x * kGroups) {
+        const long long tok = tok0 + (threadIdx.x & 31) / G;
+        const bool valid = tok < n_tok;
+        const int b = valid ? (int)(tok / p.T) : 0;
+        const int t = valid ? (int)(tok - (long long)b * p.T) : 0;
+        float c[8], s[8];
+        prologue_angles(t, rev + 8 * j, c, s);
+        // the token's head 0; head h sits h head strides further
+        const __nv_bfloat16* xt = xb + (long long)b * xs.b + (long long)t * xs.t + 8 * j;
+        __nv_bfloat16* yt = yb + (long long)b * ys.b + (long long)t * ys.t + 8 * j;
+        for (int h0 = 0; h0 < p.H; h0 += UH) {
+            uint4 ra[UH], rb[UH];
+#pragma unroll
+            for (int u = 0; u < UH; ++u) {
+                ra[u] = rb[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (valid && h0 + u < p.H) {
+                    const __nv_bfloat16* x = xt + (long long)(h0 + u) * xs.h;
+                    ra[u] = *reinterpret_cast<const uint4*>(x);
+                    rb[u] = *reinterpret_cast<const uint4*>(x + H2);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < UH; ++u) {
+                float a[8], bb[8];
+                unpack_bf16x8(ra[u], a);
+                unpack_bf16x8(rb[u], bb);
+                float inv = 1.f;
+                if (p.norm) {
+                    float ss = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss = fmaf(a[e], a[e], fmaf(bb[e], bb[e], ss));
+                    inv = 1.f / fmaxf(sqrtf(group_sum<G>(ss)), 1e-12f);
+                }
+                uint32_t oa[4], ob[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const float u0 = a[e] * inv, w0 = bb[e] * inv, u1 = a[e + 1] * inv, w1 = bb[e + 1] * inv;
+                    oa[e >> 1] = pack_bf16x2(u0 * c[e] - w0 * s[e], u1 * c[e + 1] - w1 * s[e + 1]);
+                    ob[e >> 1] = pack_bf16x2(u0 * s[e] + w0 * c[e], u1 * s[e + 1] + w1 * c[e + 1]);
+                }
+                if (valid && h0 + u < p.H) {
+                    __nv_bfloat16* y = yt + (long long)(h0 + u) * ys.h;
+                    *reinterpret_cast<uint4*>(y) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+                    *reinterpret_cast<uint4*>(y + H2) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+                }
+            }
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPrologueThreads, 4)
+qk_prologue_bwd_tok_kernel(const PrologueParams p) {
+    constexpr int G = D / 16, H2 = D / 2, kGroups = kPrologueThreads / G;
+    const int which = blockIdx.y;
+    const int j = threadIdx.x % G;
+    __shared__ double rev[D / 2];
+    prologue_rev_per_token<D>(p.base, rev);
+    const __nv_bfloat16* xb = p.x[which];
+    const __nv_bfloat16* gb = p.dy[which];
+    __nv_bfloat16* db = p.out[which];
+    const Strides xs = p.xs[which], gs = p.dys[which], ds = p.outs[which];
+    const long long n_tok = p.rows / p.H;
+    for (long long tok0 = (long long)blockIdx.x * kGroups + (threadIdx.x & ~31) / G; tok0 < n_tok;
+         tok0 += (long long)gridDim.x * kGroups) {
+        const long long tok = tok0 + (threadIdx.x & 31) / G;
+        const bool valid = tok < n_tok;
+        const int b = valid ? (int)(tok / p.T) : 0;
+        const int t = valid ? (int)(tok - (long long)b * p.T) : 0;
+        float c[8], s[8];
+        prologue_angles(t, rev + 8 * j, c, s);
+        const __nv_bfloat16* gt = gb + (long long)b * gs.b + (long long)t * gs.t + 8 * j;
+        const __nv_bfloat16* xt = xb + (long long)b * xs.b + (long long)t * xs.t + 8 * j;
+        __nv_bfloat16* dt = db + (long long)b * ds.b + (long long)t * ds.t + 8 * j;
+        for (int h = 0; h < p.H; ++h) {
+            float ga[8] = {}, gb2[8] = {}, xa[8] = {}, xb2[8] = {};
+            if (valid) {
+                const __nv_bfloat16* g = gt + (long long)h * gs.h;
+                load_bf16x8(g, ga);
+                load_bf16x8(g + H2, gb2);
+                if (p.norm) {
+                    const __nv_bfloat16* x = xt + (long long)h * xs.h;
+                    load_bf16x8(x, xa);
+                    load_bf16x8(x + H2, xb2);
+                }
+            }
+            float da[8], db2[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {            // rotate back: dn = R^T dy
+                da[e] = ga[e] * c[e] + gb2[e] * s[e];
+                db2[e] = -ga[e] * s[e] + gb2[e] * c[e];
+            }
+            if (p.norm) {
+                float ss = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss = fmaf(xa[e], xa[e], fmaf(xb2[e], xb2[e], ss));
+                const float r = sqrtf(group_sum<G>(ss));
+                const float inv = r > 1e-12f ? 1.f / r : 0.f;
+                float nd = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) nd = fmaf(xa[e], da[e], fmaf(xb2[e], db2[e], nd));
+                nd = group_sum<G>(nd) * inv;
+                if (r > 1e-12f) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        da[e] = (da[e] - xa[e] * inv * nd) * inv;
+                        db2[e] = (db2[e] - xb2[e] * inv * nd) * inv;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        da[e] *= 1e12f;
+                        db2[e] *= 1e12f;
+                    }
+                }
+            }
+            if (valid) {
+                __nv_bfloat16* d = dt + (long long)h * ds.h;
+                store_bf16x8(d, da);
+                store_bf16x8(d + H2, db2);
+            }
+        }
+    }
+}
+
 }  // namespace gpt_attn

@@ -24,16 +24,23 @@ def _err(got, ref):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("layout", ["fused", "bhtd"])
 @pytest.mark.parametrize("B,H,T,D,norm,base", [(2, 12, 1000, 64, True, 10000.0), (1, 6, 8192, 128, True, 10000.0),
                                                (2, 4, 300, 64, False, 10000.0), (2, 4, 300, 128, True, 0.0)])
-def test_prologue_then_attention_matches_oracle(B, H, T, D, norm, base):
+def test_prologue_then_attention_matches_oracle(B, H, T, D, norm, base, layout):
+    """layout "fused": q, k as views of a [B, T, 3, H, D] projection (a token's heads adjacent: the
+    kernels take a token at a time); "bhtd": contiguous [B, H, T, D] (the kernels take a row at a
+    time)."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from causal_attention_sdpa_b200 import build
     build.build()
     q, k, v, do = make_inputs(B, H, T, D, seed=T + D)
-    qkv = torch.stack([q, k, v], dim=2).permute(0, 3, 2, 1, 4).contiguous().cuda()     # [B, T, 3, H, D]
-    qr, kr, vr = (qkv[:, :, i].permute(0, 2, 1, 3) for i in range(3))
+    if layout == "fused":
+        qkv = torch.stack([q, k, v], dim=2).permute(0, 3, 2, 1, 4).contiguous().cuda()     # [B, T, 3, H, D]
+        qr, kr, vr = (qkv[:, :, i].permute(0, 2, 1, 3) for i in range(3))
+    else:
+        qr, kr, vr = q.cuda(), k.cuda(), v.cuda()
     qn, kn = ga.gpt_attn_qk_prologue_fwd(qr, kr, qk_norm=norm, rope_base=base)
     # the prologue against the oracle on the same raw rows
     for got, raw in ((qn, q), (kn, k)):
@@ -43,8 +50,11 @@ def test_prologue_then_attention_matches_oracle(B, H, T, D, norm, base):
     s = 1.0 / math.sqrt(D)
     o, lse = ga.gpt_attn_fwd(qn, kn, vr.contiguous(), scale=s)
     dq, dk, dv = ga.gpt_attn_bwd(qn, kn, vr.contiguous(), o, lse, do.cuda(), scale=s)
-    g = torch.full((B, T, 3, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
-    dqr, dkr = (g[:, :, i].permute(0, 2, 1, 3) for i in range(2))
+    if layout == "fused":
+        g = torch.full((B, T, 3, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        dqr, dkr = (g[:, :, i].permute(0, 2, 1, 3) for i in range(2))
+    else:
+        dqr, dkr = (torch.full((B, H, T, D), float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(2))
     ga.gpt_attn_qk_prologue_bwd(qr, kr, dq, dk, qk_norm=norm, rope_base=base, dq_raw=dqr, dk_raw=dkr)
     assert ga.gpt_attn_check() == ga.GPT_ATTN_OK
     for got, raw, dy in ((dqr, q, dq), (dkr, k, dk)):
