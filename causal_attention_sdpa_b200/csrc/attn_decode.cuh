@@ -47,8 +47,10 @@ __device__ __forceinline__ void decode_range(const DecodeParams& p, int bh, int&
     lo = (p.window > 0 && L - p.window > 0) ? L - p.window : 0;
 }
 
+constexpr int kDecodeBlocksPerSm = 6;     // resident split CTAs per SM (registers capped to fit)
+
 template <int D>
-__global__ void __launch_bounds__(kDecodeThreads)
+__global__ void __launch_bounds__(kDecodeThreads, kDecodeBlocksPerSm)
 attn_decode_split_kernel(const DecodeParams p) {
     constexpr int G = D / 8;                          // threads per row, 8 elements (16 bytes) each
     constexpr int R = kDecodeThreads / G;             // rows handled at once
@@ -83,7 +85,7 @@ attn_decode_split_kernel(const DecodeParams p) {
     // kU rows in flight (HBM latency is hidden by loads in flight, not by threads alone).  Every
     // thread runs the same number of iterations (rows past the chunk are predicated off), so the
     // whole warp takes part in every shuffle.
-    constexpr int kU = 8;
+    constexpr int kU = 12;
     float mloc = -INFINITY;
     for (int base = 0; base < n; base += kU * R) {
         uint4 raw[kU];
@@ -137,7 +139,7 @@ attn_decode_split_kernel(const DecodeParams p) {
     for (int w = 0; w < kDecodeThreads / 32; ++w) l += red[w];
     // o = sum_j p_j V_j: G threads per value row, R rows at once (kV of them in flight per
     // thread), then a sum over the R groups
-    constexpr int kV = 4;
+    constexpr int kV = 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int base = 0; base < n; base += kV * R) {
         uint4 raw[kV];

@@ -383,11 +383,14 @@ int check_ws(int B, int H, int T, int D, const void* ws, size_t ws_bytes) {
     return misaligned(ws) ? GPT_ATTN_ERR_ALIGN : GPT_ATTN_OK;
 }
 
-// Decode split: aim for four CTAs per SM of a B200 (148 SMs) over all heads, at least 64 keys
-// per split, at most kDecodeMaxChunk.  The same function sizes the workspace and the launch.
+// Decode split: as many splits per head as fit all CTAs on a B200 (148 SMs, kDecodeBlocksPerSm
+// resident each) in one wave, at least one, at least 64 keys per split, at most kDecodeMaxChunk.
+// A CTA's passes over its keys and values are chains of dependent load rounds, so shorter chunks
+// over more CTAs keep more of HBM busy, and a second wave would add a whole chain.  The same
+// function sizes the workspace and the launch.
 int decode_splits(int BH, int T_max, int window, int* chunk) {
     const int span = (window > 0 && window < T_max) ? window : T_max;   // keys one query can see
-    int n = (4 * 148 + BH - 1) / BH;
+    int n = kDecodeBlocksPerSm * 148 / BH;
     const int by_len = (span + 63) / 64;
     if (n > by_len) n = by_len;
     if (n < 1) n = 1;

@@ -26,6 +26,7 @@ CASES = [
     (2, 4, 8192, 128, 1024, [8192, 3000], 0.12),         # long cache, window
     (3, 2, 500, 128, 0, [0, 499, 10000], 0.088),         # empty sequence, length past the cache
     (64, 12, 1024, 64, 0, None, 0.125),                  # many heads: one split each
+    (32, 12, 1024, 64, 0, None, 0.125),                  # two splits each
 ]
 
 
